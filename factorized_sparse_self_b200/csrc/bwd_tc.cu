@@ -1,0 +1,466 @@
+// Backward pass on the tensor cores (sm_100a), with the attention matrix
+// recomputed from LSE rather than stored (milestone page "Sparse Transformer",
+// nlp-lineage, "The idea", "Recomputation").
+//
+// Per live tile pair (key tile j held by the CTA, query tile i streamed):
+//   S^T  = K Q^T                  (M=128 keys, N=128 queries, K=64)
+//   dP^T = V dO^T
+//   P^T  = exp(scale S^T - LSE_i) on the live pairs, 0 elsewhere
+//   dS^T = P^T (dP^T - D_i),      D_i = dO_i . O_i (prologue kernel)
+//   dV  += P^T dO                 (M=128, N=64, K=128)
+//   dK  += dS^T Q
+//   dQ_i = dS K  -> TMA reduce-add into the fp32 dQ accumulator
+// dV and dK stay in TMEM for the whole key tile and are reduced into fp32
+// accumulators at the end (a key tile can belong to two segments of a merged
+// head); an epilogue kernel applies the scale and rounds to bf16.
+//
+// Warp roles: warp 0 TMA producer (K, V once; Q, dO per query tile into a
+// 2-stage ring, with LSE and D by plain loads); warp 1 TMEM owner and MMA
+// issuer; warps 2..5 compute (thread = key row = TMEM lane for S^T / dP^T,
+// and query row for draining dQ). The MMA warp issues S, dP of the next tile
+// before dV, dK, dQ of the current one, so the exponentials overlap the
+// tensor pipe. All waits are bounded.
+#include <math.h>
+
+#include "launch.h"
+#include "tc_common.cuh"
+
+namespace st {
+namespace {
+
+using namespace tc;
+
+constexpr int NS = 2;
+constexpr int kTileBytes = kTile * 64 * 2;  // 128 x 64 bf16 = 16 KB
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdMaps {
+  CUtensorMap q[3], k[3], v[3], dout[3];  // bf16, indexed by View
+  CUtensorMap dq[3], dk[3], dv[3];        // fp32 accumulators, 32-float boxes
+};
+
+struct SmemBwd {
+  uint8_t k[kTileBytes];
+  uint8_t v[kTileBytes];
+  uint8_t q[NS][kTileBytes];
+  uint8_t dout[NS][kTileBytes];
+  uint8_t pt[2 * kTileBytes];    // P^T (keys x queries), two 64-query K-blocks
+  uint8_t dst[2 * kTileBytes];   // dS^T, same layout
+  uint8_t stage[2 * kTileBytes]; // fp32 dQ tile for the reduce: two 32-column halves
+  float l2[NS][kTile];           // LSE_i * log2(e) of the stage's query rows
+  float dd[NS][kTile];           // D_i
+  uint64_t kv_full, full[NS], empty[NS];
+  uint64_t s_full, dp_full, ds_ready, pds_free, dq_full, dq_free, stg_full, stg_free;
+  uint64_t kv_done, out_full, fin;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void load_tile(void* dst, const CUtensorMap* maps, int view,
+                                          const Geom& g, int tile, int bh, uint64_t* bar) {
+  if (view == VIEW_NAT) {
+    tma_load_3d(dst, &maps[VIEW_NAT], bar, 0, tile * kTile, bh);
+  } else if (view == VIEW_SUM) {
+    tma_load_4d(dst, &maps[VIEW_SUM], bar, 0, g.l - g.c, tile * (kTile / g.c), bh);
+  } else {
+    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+    tma_load_4d(dst, &maps[VIEW_CLS], bar, 0, r, pb * kTile, bh);
+  }
+}
+
+// Reduce-adds a 128-row fp32 tile, staged as two 32-column halves.
+__device__ __forceinline__ void reduce_tile(const CUtensorMap* maps, int view, const Geom& g,
+                                            int tile, int bh, const uint8_t* src) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint8_t* s = src + h * kTileBytes;
+    if (view == VIEW_NAT) {
+      tma_reduce_add_3d(&maps[VIEW_NAT], s, h * 32, tile * kTile, bh);
+    } else if (view == VIEW_SUM) {
+      tma_reduce_add_4d(&maps[VIEW_SUM], s, h * 32, g.l - g.c, tile * (kTile / g.c), bh);
+    } else {
+      int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+      tma_reduce_add_4d(&maps[VIEW_CLS], s, h * 32, r, pb * kTile, bh);
+    }
+  }
+}
+
+// Live query columns [lo, hi) of a query tile for the key at natural
+// position j (segment rules restated as intervals over queries).
+__device__ __forceinline__ void live_rows(const Geom& g, int kview, int qview, int rule,
+                                          int qtile, int j, int& lo, int& hi) {
+  if (j < 0) {
+    lo = hi = 0;
+    return;
+  }
+  const int l = g.l, c = g.c;
+  int a = 0, b = 0, base, lim;
+  if (qview == VIEW_NAT) {
+    base = qtile * kTile;
+    lim = g.T;
+    if (kview == VIEW_SUM) {
+      a = (rule == RULE_SUMMARY) ? j : (j / l + 1) * l;
+      b = lim;
+    } else {
+      switch (rule) {
+        case RULE_CAUSAL: a = j; b = lim; break;
+        case RULE_BAND: a = j; b = j + l + 1; break;
+        case RULE_BLOCK: a = j; b = (j / l + 1) * l; break;
+        case RULE_STRIDE: a = j; b = j + 1; break;                          // l >= T only
+        case RULE_SUMMARY: a = j; b = (j % l >= l - c) ? lim : j; break;    // l >= T only
+        default: a = 0; b = 0; break;
+      }
+    }
+  } else {
+    base = (qtile % g.ptiles) * kTile;
+    lim = g.P;
+    const int pk = j / l;
+    a = (rule == RULE_STRIDE) ? pk : pk + 2;
+    b = lim;
+  }
+  b = min(b, lim);
+  lo = max(a - base, 0);
+  hi = min(b - base, kTile);
+  if (hi < lo) hi = lo;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __restrict__ items,
+              const QEnt* __restrict__ qents, int B, int H, int nclasses, float scale_log2,
+              const float* __restrict__ lse, const float* __restrict__ Dg, int* status,
+              uint64_t wait_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemBwd& S = *reinterpret_cast<SmemBwd*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const BwdItem it = items[blockIdx.y];
+  const int bh = head_of(blockIdx.x, it.hclass, B, H, nclasses);
+  if (bh < 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = it.qend - it.qbeg;
+  volatile int* abort = &S.abort;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&S.kv_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&S.full[s], 33);  // expect_tx arrive + 32 producer lanes
+      mbar_init(&S.empty[s], 1);
+    }
+    mbar_init(&S.s_full, 1);
+    mbar_init(&S.dp_full, 1);
+    mbar_init(&S.ds_ready, 128);
+    mbar_init(&S.pds_free, 1);
+    mbar_init(&S.dq_full, 1);
+    mbar_init(&S.dq_free, 128);
+    mbar_init(&S.stg_full, 128);
+    mbar_init(&S.stg_free, 1);
+    mbar_init(&S.kv_done, 1);
+    mbar_init(&S.out_full, 128);
+    mbar_init(&S.fin, 1);
+    S.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  auto fail = [&]() {
+    *abort = 1;
+    set_status(status, ST_ERR_DEVICE_TIMEOUT);
+  };
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    int issued[NS] = {-1, -1};
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&S.kv_full, 2 * kTileBytes);
+      load_tile(S.k, maps.k, it.kview, g, it.ktile, bh, &S.kv_full);
+      load_tile(S.v, maps.v, it.kview, g, it.ktile, bh, &S.kv_full);
+    }
+    for (int e = 0; e < n; ++e) {
+      const int s = e % NS;
+      if (e >= NS) {
+        bool ok = mbar_wait(&S.empty[s], ((e / NS) - 1) & 1, wait_ns, abort);
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) fail();
+          break;
+        }
+      }
+      const QEnt qe = qents[it.qbeg + e];
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&S.full[s], 2 * kTileBytes);
+        load_tile(S.q[s], maps.q, it.qview, g, qe.qtile, bh, &S.full[s]);
+        load_tile(S.dout[s], maps.dout, it.qview, g, qe.qtile, bh, &S.full[s]);
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int row = lane + 32 * t;
+        const int i = view_pos(g, it.qview, qe.qtile, row);
+        S.l2[s][row] = (i >= 0) ? lse[(size_t)bh * g.T + i] * kLog2e : 0.f;
+        S.dd[s][row] = (i >= 0) ? Dg[(size_t)bh * g.T + i] : 0.f;
+      }
+      mbar_arrive(&S.full[s]);
+      issued[s] = e;
+    }
+    if (lane == 0) {
+      mbar_wait(&S.kv_full, 0, wait_ns, abort);
+      for (int s = 0; s < NS; ++s)
+        if (issued[s] >= 0 && !mbar_wait(&S.full[s], (issued[s] / NS) & 1, wait_ns, abort))
+          fail();
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idSS = idesc_bf16(128, 128, false, false);
+      const uint32_t idKM = idesc_bf16(128, 64, false, true);  // A K-major, B MN-major
+      const uint32_t idMM = idesc_bf16(128, 64, true, true);   // A MN-major, B MN-major
+      const uint32_t k_addr = smem_u32(S.k), v_addr = smem_u32(S.v);
+      const uint32_t pt_addr = smem_u32(S.pt), ds_addr = smem_u32(S.dst);
+      bool ok = mbar_wait(&S.kv_full, 0, wait_ns, abort);
+      auto issue_s_dp = [&](int e) -> bool {
+        const int s = e % NS;
+        if (!mbar_wait(&S.full[s], (e / NS) & 1, wait_ns, abort)) return false;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(S.q[s]), o_addr = smem_u32(S.dout[s]);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem + kColS, sdesc(k_addr + kk * 32, 16, 1024), sdesc(q_addr + kk * 32, 16, 1024),
+                 idSS, kk > 0);
+        mma_commit(&S.s_full);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem + kColDP, sdesc(v_addr + kk * 32, 16, 1024),
+                 sdesc(o_addr + kk * 32, 16, 1024), idSS, kk > 0);
+        mma_commit(&S.dp_full);
+        return true;
+      };
+      if (ok) ok = issue_s_dp(0);
+      for (int e = 0; ok && e < n; ++e) {
+        const int s = e % NS;
+        if (!mbar_wait(&S.ds_ready, e & 1, wait_ns, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (e + 1 < n && !issue_s_dp(e + 1)) {
+          ok = false;
+          break;
+        }
+        const uint32_t q_addr = smem_u32(S.q[s]), o_addr = smem_u32(S.dout[s]);
+        // dV += P^T dO ; dK += dS^T Q   (K = 128 queries, 8 steps of 16)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + kColDV, sdesc(pt_addr + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
+                 sdesc(o_addr + kk * 2048, 16384, 1024), idKM, (e > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + kColDK, sdesc(ds_addr + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
+                 sdesc(q_addr + kk * 2048, 16384, 1024), idKM, (e > 0 || kk > 0) ? 1u : 0u);
+        if (e > 0 && !mbar_wait(&S.dq_free, (e - 1) & 1, wait_ns, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // dQ = dS K   (A = dS^T read MN-major, K = 128 keys)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + kColDQ, sdesc(ds_addr + kk * 2048, kTileBytes, 1024),
+                 sdesc(k_addr + kk * 2048, 16384, 1024), idMM, kk > 0 ? 1u : 0u);
+        mma_commit(&S.dq_full);
+        mma_commit(&S.pds_free);
+        mma_commit(&S.empty[s]);
+      }
+      if (!ok) fail();
+      mma_commit(&S.kv_done);
+      mma_commit(&S.fin);
+      mbar_wait(&S.fin, 0, wait_ns, abort);
+    }
+  } else {
+    // ---------------- compute warps ----------------
+    const int lg = warp & 3;
+    const int row = lg * 32 + lane;               // key row (S^T, dP^T) / query row (dQ)
+    const uint32_t tl = (uint32_t)(lg * 32) << 16;
+    const int j = view_pos(g, it.kview, it.ktile, row);
+    const bool issuer = (warp == 2 && lane == 0);
+    bool ok = true;
+    const uint32_t pt_addr = smem_u32(S.pt), ds_addr = smem_u32(S.dst), st_addr = smem_u32(S.stage);
+
+    // dQ of tile e: TMEM -> registers -> fp32 staging -> TMA reduce-add
+    auto drain_dq = [&](int e) -> bool {
+      bool w = mbar_wait(&S.dq_full, e & 1, wait_ns, abort);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      uint32_t dq[64];
+      tmem_ld32(tmem + tl + kColDQ, dq);
+      tmem_ld32(tmem + tl + kColDQ + 32, dq + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&S.dq_free);
+      if (e > 0) {
+        w = mbar_wait(&S.stg_free, (e - 1) & 1, wait_ns, abort);
+        if (!__all_sync(0xffffffffu, w)) return false;
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          st_shared_v4(st_addr + h * kTileBytes + swz128(row, ch), dq[h * 32 + ch * 4 + 0],
+                       dq[h * 32 + ch * 4 + 1], dq[h * 32 + ch * 4 + 2], dq[h * 32 + ch * 4 + 3]);
+      fence_async_smem();
+      mbar_arrive(&S.stg_full);
+      if (issuer) {
+        if (!mbar_wait(&S.stg_full, e & 1, wait_ns, abort)) return false;
+        const QEnt qe = qents[it.qbeg + e];
+        reduce_tile(maps.dq, it.qview, g, qe.qtile, bh, S.stage);
+        bulk_commit();
+        bulk_wait_read_all();
+        mbar_arrive(&S.stg_free);
+      }
+      return true;
+    };
+
+    for (int e = 0; e < n; ++e) {
+      const int s = e % NS;
+      const QEnt qe = qents[it.qbeg + e];
+      bool w = mbar_wait(&S.s_full, e & 1, wait_ns, abort);
+      w = w && mbar_wait(&S.dp_full, e & 1, wait_ns, abort);
+      w = w && mbar_wait(&S.full[s], (e / NS) & 1, wait_ns, abort);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      int lo = 0, hi = kTile;
+      if (qe.flag != TILE_FULL) live_rows(g, it.kview, it.qview, it.rule, qe.qtile, j, lo, hi);
+      if (e > 0) {
+        w = mbar_wait(&S.pds_free, (e - 1) & 1, wait_ns, abort);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+      }
+      const float* l2 = S.l2[s];
+      const float* dd = S.dd[s];
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float sv[64], dp[64];
+        tmem_ld32(tmem + tl + kColS + h * 64, reinterpret_cast<uint32_t*>(sv));
+        tmem_ld32(tmem + tl + kColS + h * 64 + 32, reinterpret_cast<uint32_t*>(sv) + 32);
+        tmem_ld32(tmem + tl + kColDP + h * 64, reinterpret_cast<uint32_t*>(dp));
+        tmem_ld32(tmem + tl + kColDP + h * 64 + 32, reinterpret_cast<uint32_t*>(dp) + 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t pw[4], dw[4];
+#pragma unroll
+          for (int x2 = 0; x2 < 4; ++x2) {
+            float pv[2], dv2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int x = ch * 8 + x2 * 2 + u;   // column within this half
+              const int col = h * 64 + x;          // query column in the tile
+              const bool live = (col >= lo) && (col < hi);
+              const float p = live ? fast_exp2(fmaf(sv[x], scale_log2, -l2[col])) : 0.f;
+              pv[u] = p;
+              dv2[u] = p * (dp[x] - dd[col]);
+            }
+            pw[x2] = pack_bf16(pv[0], pv[1]);
+            dw[x2] = pack_bf16(dv2[0], dv2[1]);
+          }
+          st_shared_v4(pt_addr + h * kTileBytes + swz128(row, ch), pw[0], pw[1], pw[2], pw[3]);
+          st_shared_v4(ds_addr + h * kTileBytes + swz128(row, ch), dw[0], dw[1], dw[2], dw[3]);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&S.ds_ready);
+      if (e > 0 && !drain_dq(e - 1)) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok && n > 0 && !drain_dq(n - 1)) ok = false;
+    if (ok) {
+      // dK, dV of this key tile: TMEM -> fp32 staging (P^T, dS^T buffers) -> reduce-add
+      bool w = mbar_wait(&S.kv_done, 0, wait_ns, abort);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+      } else {
+        tc_fence_after();
+        uint32_t r[64];
+        tmem_ld32(tmem + tl + kColDK, r);
+        tmem_ld32(tmem + tl + kColDK + 32, r + 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            st_shared_v4(pt_addr + h * kTileBytes + swz128(row, ch), r[h * 32 + ch * 4 + 0],
+                         r[h * 32 + ch * 4 + 1], r[h * 32 + ch * 4 + 2], r[h * 32 + ch * 4 + 3]);
+        tmem_ld32(tmem + tl + kColDV, r);
+        tmem_ld32(tmem + tl + kColDV + 32, r + 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            st_shared_v4(ds_addr + h * kTileBytes + swz128(row, ch), r[h * 32 + ch * 4 + 0],
+                         r[h * 32 + ch * 4 + 1], r[h * 32 + ch * 4 + 2], r[h * 32 + ch * 4 + 3]);
+        fence_async_smem();
+        mbar_arrive(&S.out_full);
+        if (issuer) {
+          if (mbar_wait(&S.out_full, 0, wait_ns, abort)) {
+            reduce_tile(maps.dk, it.kview, g, it.ktile, bh, S.pt);
+            reduce_tile(maps.dv, it.kview, g, it.ktile, bh, S.dst);
+            bulk_commit();
+          } else {
+            ok = false;
+          }
+        }
+      }
+    }
+    if (!ok) fail();
+    if (issuer) bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+}  // namespace st
+
+namespace st {
+
+cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, const float* lse,
+                   const void* dout, const float* D, float* dq_acc, float* dk_acc,
+                   float* dv_acc) {
+  const st_layout* L = c.L;
+  const int BH = c.B * c.H;
+  if (L->dev.n_bwd_items == 0) return cudaSuccess;
+  BwdMaps maps;
+  if (!make_view_maps(maps.q, q, false, L->geom, BH, c.d) ||
+      !make_view_maps(maps.k, k, false, L->geom, BH, c.d) ||
+      !make_view_maps(maps.v, v, false, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dout, dout, false, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dq, dq_acc, true, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dk, dk_acc, true, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dv, dv_acc, true, L->geom, BH, c.d))
+    return cudaErrorInvalidValue;
+  const size_t smem = sizeof(SmemBwd) + 1024;
+  cudaError_t err =
+      cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  dim3 grid(heads_per_class(c), L->dev.n_bwd_items);
+  bwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
+      maps, L->geom, (const BwdItem*)L->dev.bwd_items, (const QEnt*)L->dev.q_ents, c.B, c.H,
+      c.nclasses, c.scale * kLog2e, lse, D, c.status, c.wait_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace st

@@ -1,0 +1,83 @@
+// Device helpers shared by every kernel of the library: view-row mapping,
+// the membership rules of the segments, and the device status word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "st_internal.h"
+
+namespace st {
+
+// Natural position of row k of tile `tile` in view v; -1 for padding rows.
+__device__ __forceinline__ int view_pos(const Geom& g, int v, int tile, int k) {
+  if (v == VIEW_NAT) {
+    int t = tile * kTile + k;
+    return t < g.T ? t : -1;
+  }
+  if (v == VIEW_SUM) {
+    int s = tile * kTile + k;
+    if (s >= g.nsum) return -1;
+    return (s / g.c) * g.l + (g.l - g.c) + s % g.c;
+  }
+  int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+  int p = pb * kTile + k;
+  if (p >= g.P) return -1;
+  return p * g.l + r;
+}
+
+// Membership of the pair (i, j), natural positions, in a segment rule. The
+// rules restate the index sets: strided window / stride, fixed block /
+// summary positions ("Sparse Transformer", llm-arch-kb, section 2).
+__device__ __forceinline__ bool rule_live(const Geom& g, int rule, int i, int j) {
+  if (i < 0 || j < 0 || j > i) return false;
+  const int l = g.l, c = g.c;
+  switch (rule) {
+    case RULE_CAUSAL:
+      return true;
+    case RULE_BAND:
+      return j >= i - l;
+    case RULE_BLOCK:
+      return j / l == i / l;
+    case RULE_STRIDE:
+      return (i - j) % l == 0;
+    case RULE_STRIDE_FAR:
+      return (i - j) % l == 0 && i - j >= 2 * l;
+    case RULE_SUMMARY:
+      return j % l >= l - c;
+    case RULE_SUMMARY_EARLIER:
+      return j % l >= l - c && j / l < i / l;
+    default:
+      return false;
+  }
+}
+
+// Head index bh = b*H + h of grid column x for a head class: split mode puts
+// even heads in class 0 and odd heads in class 1. Returns -1 past the end.
+__device__ __forceinline__ int head_of(int x, int hclass, int B, int H, int nclasses) {
+  if (nclasses == 1) return x < B * H ? x : -1;
+  int per = (hclass == 0) ? (H + 1) / 2 : H / 2;
+  if (per == 0 || x >= B * per) return -1;
+  int b = x / per, hh = x - b * per;
+  return b * H + 2 * hh + hclass;
+}
+
+__device__ __forceinline__ void set_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <class T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+}  // namespace st

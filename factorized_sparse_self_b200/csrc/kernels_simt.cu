@@ -1,0 +1,407 @@
+// Exact-fp32 path on CUDA cores, plus the backward prologue and epilogue.
+//
+// The fp32 kernels walk the same schedule as the tensor-core kernels (work
+// items of 128-row query or key tiles, each with its live tiles) and test
+// membership with the segment rules on PARTIAL tiles. They exist for float32
+// inputs, whose tolerance leaves no room for reduced-precision tensor-core
+// arithmetic; one thread owns one query (forward, dQ) or one key (dK, dV).
+//
+// Attention over an allowed set and its normalisation: "Sparse Transformer"
+// milestone page (nlp-lineage), "The notation"; llm-arch-kb section 2,
+// "Sparse attention as an unnormalized form". Backward with the attention
+// matrix recomputed from LSE: milestone page, "Recomputation".
+#include <math.h>
+
+#include "device_common.cuh"
+#include "launch.h"
+
+namespace st {
+namespace {
+
+constexpr int kThreads = 128;
+
+template <int D>
+__device__ __forceinline__ float dot_smem(const float* a, const float* b) {
+  float s = 0.f;
+#pragma unroll
+  for (int x = 0; x < D; ++x) s = fmaf(a[x], b[x], s);
+  return s;
+}
+
+// smem: Ks[128][D+1], Vs[128][D+1], jpos[128]
+template <class E, int D>
+__global__ void __launch_bounds__(kThreads)
+simt_fwd_kernel(Geom g, const FwdItem* __restrict__ items, const KeyEnt* __restrict__ keys,
+                int B, int H, int nclasses, float scale, const E* __restrict__ q,
+                const E* __restrict__ k, const E* __restrict__ v, E* __restrict__ o,
+                float* __restrict__ lse) {
+  extern __shared__ float sm[];
+  float* Ks = sm;
+  float* Vs = Ks + kTile * (D + 1);
+  int* jpos = reinterpret_cast<int*>(Vs + kTile * (D + 1));
+  const FwdItem it = items[blockIdx.y];
+  const int bh = head_of(blockIdx.x, it.hclass, B, H, nclasses);
+  if (bh < 0) return;
+  const size_t base = (size_t)bh * g.T * D;
+  const int tid = threadIdx.x;
+  const int i = view_pos(g, it.qview, it.qtile, tid);
+  float qr[D], acc[D];
+#pragma unroll
+  for (int x = 0; x < D; ++x) {
+    qr[x] = (i >= 0) ? to_f32(q[base + (size_t)i * D + x]) * scale : 0.f;
+    acc[x] = 0.f;
+  }
+  float m = -INFINITY, lsum = 0.f;
+  for (int e = it.kbeg; e < it.kend; ++e) {
+    const KeyEnt ke = keys[e];
+    __syncthreads();
+    for (int idx = tid; idx < kTile * D; idx += kThreads) {
+      int r = idx / D, x = idx - r * D;
+      int j = view_pos(g, ke.kview, ke.ktile, r);
+      Ks[r * (D + 1) + x] = (j >= 0) ? to_f32(k[base + (size_t)j * D + x]) : 0.f;
+      Vs[r * (D + 1) + x] = (j >= 0) ? to_f32(v[base + (size_t)j * D + x]) : 0.f;
+    }
+    jpos[tid] = view_pos(g, ke.kview, ke.ktile, tid);
+    __syncthreads();
+    if (i < 0) continue;
+    for (int r = 0; r < kTile; ++r) {
+      const int j = jpos[r];
+      if (j < 0) continue;
+      if (ke.flag != TILE_FULL && !rule_live(g, ke.rule, i, j)) continue;
+      const float s = dot_smem<D>(qr, Ks + r * (D + 1));
+      if (s > m) {
+        const float corr = expf(m - s);
+        lsum *= corr;
+#pragma unroll
+        for (int x = 0; x < D; ++x) acc[x] *= corr;
+        m = s;
+      }
+      const float p = expf(s - m);
+      lsum += p;
+      const float* vr = Vs + r * (D + 1);
+#pragma unroll
+      for (int x = 0; x < D; ++x) acc[x] = fmaf(p, vr[x], acc[x]);
+    }
+  }
+  if (i < 0) return;
+  float L = (lsum > 0.f) ? m + logf(lsum) : -INFINITY;
+  float w_cur = (lsum > 0.f) ? 1.f / lsum : 0.f;
+  float w_prev = 0.f;
+  const size_t orow = base + (size_t)i * D;
+  if (it.merge) {
+    const float Lp = lse[(size_t)bh * g.T + i];
+    const float mx = fmaxf(Lp, L);
+    if (mx == -INFINITY) {
+      L = -INFINITY;
+      w_cur = 0.f;
+    } else {
+      const float ep = expf(Lp - mx), ec = expf(L - mx);
+      const float Ln = mx + logf(ep + ec);
+      w_prev = expf(Lp - Ln);
+      w_cur *= expf(L - Ln);
+      L = Ln;
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < D; ++x) {
+    float val = acc[x] * w_cur;
+    if (it.merge) val = fmaf(w_prev, to_f32(o[orow + x]), val);
+    o[orow + x] = from_f32<E>(val);
+  }
+  lse[(size_t)bh * g.T + i] = L;
+}
+
+// Key-major dK, dV. smem: Ks, Vs (own rows), Qs, dOs [128][D+1]; lses, Ds, ipos [128].
+template <class E, int D>
+__global__ void __launch_bounds__(kThreads)
+simt_bwd_kv_kernel(Geom g, const BwdItem* __restrict__ items, const QEnt* __restrict__ qents,
+                   int B, int H, int nclasses, float scale, const E* __restrict__ q,
+                   const E* __restrict__ k, const E* __restrict__ v, const float* __restrict__ lse,
+                   const E* __restrict__ dout, const float* __restrict__ Dv,
+                   float* __restrict__ dk_acc, float* __restrict__ dv_acc) {
+  extern __shared__ float sm[];
+  float* Ks = sm;
+  float* Vs = Ks + kTile * (D + 1);
+  float* Qs = Vs + kTile * (D + 1);
+  float* dOs = Qs + kTile * (D + 1);
+  float* lses = dOs + kTile * (D + 1);
+  float* Ds = lses + kTile;
+  int* ipos = reinterpret_cast<int*>(Ds + kTile);
+  const BwdItem it = items[blockIdx.y];
+  const int bh = head_of(blockIdx.x, it.hclass, B, H, nclasses);
+  if (bh < 0) return;
+  const size_t base = (size_t)bh * g.T * D;
+  const size_t rbase = (size_t)bh * g.T;
+  const int tid = threadIdx.x;
+  const int j = view_pos(g, it.kview, it.ktile, tid);
+  float* kr = Ks + tid * (D + 1);
+  float* vr = Vs + tid * (D + 1);
+  float dk[D], dv[D];
+#pragma unroll
+  for (int x = 0; x < D; ++x) {
+    kr[x] = (j >= 0) ? to_f32(k[base + (size_t)j * D + x]) : 0.f;
+    vr[x] = (j >= 0) ? to_f32(v[base + (size_t)j * D + x]) : 0.f;
+    dk[x] = 0.f;
+    dv[x] = 0.f;
+  }
+  for (int e = it.qbeg; e < it.qend; ++e) {
+    const QEnt qe = qents[e];
+    __syncthreads();
+    for (int idx = tid; idx < kTile * D; idx += kThreads) {
+      int r = idx / D, x = idx - r * D;
+      int ii = view_pos(g, it.qview, qe.qtile, r);
+      Qs[r * (D + 1) + x] = (ii >= 0) ? to_f32(q[base + (size_t)ii * D + x]) : 0.f;
+      dOs[r * (D + 1) + x] = (ii >= 0) ? to_f32(dout[base + (size_t)ii * D + x]) : 0.f;
+    }
+    {
+      int ii = view_pos(g, it.qview, qe.qtile, tid);
+      ipos[tid] = ii;
+      lses[tid] = (ii >= 0) ? lse[rbase + ii] : 0.f;
+      Ds[tid] = (ii >= 0) ? Dv[rbase + ii] : 0.f;
+    }
+    __syncthreads();
+    if (j < 0) continue;
+    for (int r = 0; r < kTile; ++r) {
+      const int ii = ipos[r];
+      if (ii < 0) continue;
+      if (qe.flag != TILE_FULL && !rule_live(g, it.rule, ii, j)) continue;
+      const float* qr = Qs + r * (D + 1);
+      const float* dor = dOs + r * (D + 1);
+      const float s = scale * dot_smem<D>(qr, kr);
+      const float p = expf(s - lses[r]);
+      const float dp = dot_smem<D>(dor, vr);
+      const float ds = p * (dp - Ds[r]) * scale;
+#pragma unroll
+      for (int x = 0; x < D; ++x) {
+        dv[x] = fmaf(p, dor[x], dv[x]);
+        dk[x] = fmaf(ds, qr[x], dk[x]);
+      }
+    }
+  }
+  if (j < 0) return;
+#pragma unroll
+  for (int x = 0; x < D; ++x) {
+    atomicAdd(dk_acc + base + (size_t)j * D + x, dk[x]);
+    atomicAdd(dv_acc + base + (size_t)j * D + x, dv[x]);
+  }
+}
+
+// Query-major dQ over the forward schedule. smem: Ks, Vs [128][D+1], own Q and
+// dO rows [128][D+1], jpos [128].
+template <class E, int D>
+__global__ void __launch_bounds__(kThreads)
+simt_bwd_q_kernel(Geom g, const FwdItem* __restrict__ items, const KeyEnt* __restrict__ keys,
+                  int B, int H, int nclasses, float scale, const E* __restrict__ q,
+                  const E* __restrict__ k, const E* __restrict__ v,
+                  const float* __restrict__ lse, const E* __restrict__ dout,
+                  const float* __restrict__ Dv, float* __restrict__ dq_acc) {
+  extern __shared__ float sm[];
+  float* Ks = sm;
+  float* Vs = Ks + kTile * (D + 1);
+  float* Qo = Vs + kTile * (D + 1);
+  float* dOo = Qo + kTile * (D + 1);
+  int* jpos = reinterpret_cast<int*>(dOo + kTile * (D + 1));
+  const FwdItem it = items[blockIdx.y];
+  if (it.kbeg == it.kend) return;
+  const int bh = head_of(blockIdx.x, it.hclass, B, H, nclasses);
+  if (bh < 0) return;
+  const size_t base = (size_t)bh * g.T * D;
+  const int tid = threadIdx.x;
+  const int i = view_pos(g, it.qview, it.qtile, tid);
+  float* qr = Qo + tid * (D + 1);
+  float* dor = dOo + tid * (D + 1);
+  float dq[D];
+#pragma unroll
+  for (int x = 0; x < D; ++x) {
+    qr[x] = (i >= 0) ? to_f32(q[base + (size_t)i * D + x]) : 0.f;
+    dor[x] = (i >= 0) ? to_f32(dout[base + (size_t)i * D + x]) : 0.f;
+    dq[x] = 0.f;
+  }
+  const float Li = (i >= 0) ? lse[(size_t)bh * g.T + i] : 0.f;
+  const float Di = (i >= 0) ? Dv[(size_t)bh * g.T + i] : 0.f;
+  for (int e = it.kbeg; e < it.kend; ++e) {
+    const KeyEnt ke = keys[e];
+    __syncthreads();
+    for (int idx = tid; idx < kTile * D; idx += kThreads) {
+      int r = idx / D, x = idx - r * D;
+      int j = view_pos(g, ke.kview, ke.ktile, r);
+      Ks[r * (D + 1) + x] = (j >= 0) ? to_f32(k[base + (size_t)j * D + x]) : 0.f;
+      Vs[r * (D + 1) + x] = (j >= 0) ? to_f32(v[base + (size_t)j * D + x]) : 0.f;
+    }
+    jpos[tid] = view_pos(g, ke.kview, ke.ktile, tid);
+    __syncthreads();
+    if (i < 0) continue;
+    for (int r = 0; r < kTile; ++r) {
+      const int j = jpos[r];
+      if (j < 0) continue;
+      if (ke.flag != TILE_FULL && !rule_live(g, ke.rule, i, j)) continue;
+      const float* kr = Ks + r * (D + 1);
+      const float s = scale * dot_smem<D>(qr, kr);
+      const float p = expf(s - Li);
+      const float dp = dot_smem<D>(dor, Vs + r * (D + 1));
+      const float ds = p * (dp - Di);
+#pragma unroll
+      for (int x = 0; x < D; ++x) dq[x] = fmaf(ds, kr[x], dq[x]);
+    }
+  }
+  if (i < 0) return;
+#pragma unroll
+  for (int x = 0; x < D; ++x) atomicAdd(dq_acc + base + (size_t)i * D + x, dq[x] * scale);
+}
+
+// One warp per row: D_i = sum_x dout_ix * o_ix; then the accumulators are zeroed.
+template <class E>
+__global__ void prologue_kernel(const E* __restrict__ o, const E* __restrict__ dout,
+                                float* __restrict__ Dv, size_t rows, int d,
+                                float4* __restrict__ acc, size_t acc_vec) {
+  const int lane = threadIdx.x & 31;
+  const size_t warp = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5;
+  const size_t nwarps = (gridDim.x * (size_t)blockDim.x) >> 5;
+  for (size_t r = warp; r < rows; r += nwarps) {
+    float s = 0.f;
+    for (int x = lane; x < d; x += 32) s = fmaf(to_f32(dout[r * d + x]), to_f32(o[r * d + x]), s);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) Dv[r] = s;
+  }
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < acc_vec;
+       t += gridDim.x * (size_t)blockDim.x)
+    acc[t] = z;
+}
+
+// Rounds the fp32 accumulators (dQ, dK, dV back to back) into bf16 outputs;
+// dQ and dK are scaled here because the tensor-core kernel accumulates dS K
+// and dS^T Q unscaled.
+__global__ void epilogue_kernel(const float4* __restrict__ acc, __nv_bfloat162* __restrict__ dq,
+                                __nv_bfloat162* __restrict__ dk, __nv_bfloat162* __restrict__ dv,
+                                size_t vec, float scale) {
+  for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < vec;
+       t += gridDim.x * (size_t)blockDim.x) {
+    float4 a = acc[t], b = acc[vec + t], c = acc[2 * vec + t];
+    a.x *= scale; a.y *= scale; a.z *= scale; a.w *= scale;
+    b.x *= scale; b.y *= scale; b.z *= scale; b.w *= scale;
+    dq[2 * t] = __floats2bfloat162_rn(a.x, a.y);
+    dq[2 * t + 1] = __floats2bfloat162_rn(a.z, a.w);
+    dk[2 * t] = __floats2bfloat162_rn(b.x, b.y);
+    dk[2 * t + 1] = __floats2bfloat162_rn(b.z, b.w);
+    dv[2 * t] = __floats2bfloat162_rn(c.x, c.y);
+    dv[2 * t + 1] = __floats2bfloat162_rn(c.z, c.w);
+  }
+}
+
+int grid_cap(size_t work, int per_block) {
+  size_t b = (work + per_block - 1) / per_block;
+  if (b > 148 * 16) b = 148 * 16;
+  if (b < 1) b = 1;
+  return (int)b;
+}
+
+template <class E, int D>
+cudaError_t simt_fwd_t(const Call& c, const void* q, const void* k, const void* v, void* o,
+                       float* lse) {
+  const st_layout* L = c.L;
+  size_t smem = sizeof(float) * 2 * kTile * (D + 1) + sizeof(int) * kTile;
+  auto kern = simt_fwd_kernel<E, D>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+  if (err != cudaSuccess) return err;
+  for (int pass = 0; pass < L->n_passes; ++pass) {
+    int n = L->dev.n_fwd_items[pass];
+    if (n == 0) continue;
+    dim3 grid(heads_per_class(c), n);
+    kern<<<grid, kThreads, smem, c.stream>>>(
+        L->geom, (const FwdItem*)L->dev.fwd_items[pass], (const KeyEnt*)L->dev.key_ents, c.B,
+        c.H, c.nclasses, c.scale, (const E*)q, (const E*)k, (const E*)v, (E*)o, lse);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+template <class E, int D>
+cudaError_t simt_bwd_t(const Call& c, const void* q, const void* k, const void* v,
+                       const float* lse, const void* dout, const float* Dv, float* dq_acc,
+                       float* dk_acc, float* dv_acc) {
+  const st_layout* L = c.L;
+  size_t smem_kv = sizeof(float) * (4 * kTile * (D + 1) + 2 * kTile) + sizeof(int) * kTile;
+  size_t smem_q = sizeof(float) * 4 * kTile * (D + 1) + sizeof(int) * kTile;
+  auto kv = simt_bwd_kv_kernel<E, D>;
+  auto kq = simt_bwd_q_kernel<E, D>;
+  cudaError_t err =
+      cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_q);
+  if (err != cudaSuccess) return err;
+  if (L->dev.n_bwd_items > 0) {
+    dim3 grid(heads_per_class(c), L->dev.n_bwd_items);
+    kv<<<grid, kThreads, smem_kv, c.stream>>>(
+        L->geom, (const BwdItem*)L->dev.bwd_items, (const QEnt*)L->dev.q_ents, c.B, c.H,
+        c.nclasses, c.scale, (const E*)q, (const E*)k, (const E*)v, lse, (const E*)dout, Dv,
+        dk_acc, dv_acc);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  for (int pass = 0; pass < L->n_passes; ++pass) {
+    int n = L->dev.n_fwd_items[pass];
+    if (n == 0) continue;
+    dim3 grid(heads_per_class(c), n);
+    kq<<<grid, kThreads, smem_q, c.stream>>>(
+        L->geom, (const FwdItem*)L->dev.fwd_items[pass], (const KeyEnt*)L->dev.key_ents, c.B,
+        c.H, c.nclasses, c.scale, (const E*)q, (const E*)k, (const E*)v, lse, (const E*)dout,
+        Dv, dq_acc);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t simt_fwd(const Call& c, const void* q, const void* k, const void* v, void* o,
+                     float* lse) {
+  if (c.dtype == ST_F32) {
+    if (c.d == 32) return simt_fwd_t<float, 32>(c, q, k, v, o, lse);
+    if (c.d == 64) return simt_fwd_t<float, 64>(c, q, k, v, o, lse);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t simt_bwd(const Call& c, const void* q, const void* k, const void* v,
+                     const float* lse, const void* dout, const float* Dv, float* dq_acc,
+                     float* dk_acc, float* dv_acc) {
+  if (c.dtype == ST_F32) {
+    if (c.d == 32)
+      return simt_bwd_t<float, 32>(c, q, k, v, lse, dout, Dv, dq_acc, dk_acc, dv_acc);
+    if (c.d == 64)
+      return simt_bwd_t<float, 64>(c, q, k, v, lse, dout, Dv, dq_acc, dk_acc, dv_acc);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* Dv, float* acc,
+                         size_t acc_elems) {
+  size_t rows = (size_t)c.B * c.H * c.L->geom.T;
+  int threads = 256;
+  int blocks = grid_cap(rows * 32 > acc_elems / 4 ? rows * 32 : acc_elems / 4, threads);
+  if (c.dtype == ST_F32)
+    prologue_kernel<float><<<blocks, threads, 0, c.stream>>>(
+        (const float*)o, (const float*)dout, Dv, rows, c.d, (float4*)acc, acc_elems / 4);
+  else
+    prologue_kernel<__nv_bfloat16><<<blocks, threads, 0, c.stream>>>(
+        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, Dv, rows, c.d, (float4*)acc,
+        acc_elems / 4);
+  return cudaGetLastError();
+}
+
+cudaError_t bwd_epilogue(const Call& c, const float* acc, void* dq, void* dk, void* dv,
+                         size_t elems) {
+  size_t vec = elems / 4;
+  int threads = 256;
+  epilogue_kernel<<<grid_cap(vec, threads), threads, 0, c.stream>>>(
+      (const float4*)acc, (__nv_bfloat162*)dq, (__nv_bfloat162*)dk, (__nv_bfloat162*)dv, vec,
+      c.scale);
+  return cudaGetLastError();
+}
+
+}  // namespace st

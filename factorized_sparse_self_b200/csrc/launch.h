@@ -1,0 +1,59 @@
+// Host-side launch entry points of the kernels (internal; CUDA files only).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "st_internal.h"
+
+namespace st {
+
+struct Call {
+  const st_layout* L;
+  int dtype;  // st_dtype
+  int B, H, d;
+  float scale;
+  int nclasses;     // head classes of the layout
+  int* status;      // device status word
+  uint64_t wait_ns; // bound of every on-device wait
+  cudaStream_t stream;
+};
+
+// Exact fp32 path (CUDA cores): float32 tensors, d = 32 or 64.
+cudaError_t simt_fwd(const Call& c, const void* q, const void* k, const void* v, void* o,
+                     float* lse);
+cudaError_t simt_bwd(const Call& c, const void* q, const void* k, const void* v,
+                     const float* lse, const void* dout, const float* D, float* dq_acc,
+                     float* dk_acc, float* dv_acc);
+
+// Backward prologue (D_i = dout_i . O_i, zero the fp32 accumulators) and,
+// for bf16, the epilogue that rounds the accumulators into dq, dk, dv.
+cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* D, float* acc,
+                         size_t acc_elems);
+cudaError_t bwd_epilogue(const Call& c, const float* acc, void* dq, void* dk, void* dv,
+                         size_t elems);
+
+// Tensor-core path (tcgen05 + TMA): bf16, d = 64.
+cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, void* o,
+                   float* lse, int force_timeout);
+cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v,
+                   const float* lse, const void* dout, const float* D, float* dq_acc,
+                   float* dk_acc, float* dv_acc);
+
+}  // namespace st
+
+#include <cuda.h>
+
+namespace st {
+
+inline int heads_per_class(const Call& c) {
+  return c.nclasses == 1 ? c.B * c.H : c.B * ((c.H + 1) / 2);
+}
+
+// Encodes the natural (3-D), summary and residue-class (4-D) TMA views of a
+// [B*H, T, d] tensor: bf16 with 64-element boxes, or fp32 with 32-element
+// boxes; 128-byte swizzle; 128-row boxes. Views the layout lacks get a copy
+// of the natural map (never used). Returns false if the driver rejects one.
+bool make_view_maps(CUtensorMap out[3], const void* base, bool is_f32, const Geom& g, int BH,
+                    int d);
+
+}  // namespace st

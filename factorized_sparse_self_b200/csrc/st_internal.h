@@ -1,0 +1,131 @@
+// Internal declarations shared by the host layout builder and the CUDA side
+// of libsparse_transformer_attn.so. Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+#include <vector>
+
+#include "../../include/sparse_transformer_attn.h"
+
+namespace st {
+
+constexpr int kTile = 128;  // query and key tile edge, in view rows
+
+// Row orders ("views") a segment reads its queries or keys in.
+enum View : uint8_t {
+  VIEW_NAT = 0,  // natural order, position t
+  VIEW_SUM = 1,  // summary keys: sigma = floor(j/l)*c + (j mod l) - (l-c)
+  VIEW_CLS = 2,  // residue class r = t mod l, row p = floor(t/l); tiles never
+                 // straddle classes (each class padded to a multiple of 128)
+};
+
+// Membership rule of a segment, in natural coordinates (all imply j <= i).
+enum Rule : uint8_t {
+  RULE_CAUSAL = 0,          // every j <= i
+  RULE_BAND = 1,            // i - l <= j                       (strided A1)
+  RULE_BLOCK = 2,           // floor(j/l) == floor(i/l)         (fixed A1)
+  RULE_STRIDE = 3,          // (i - j) mod l == 0               (strided A2)
+  RULE_STRIDE_FAR = 4,      // (i - j) mod l == 0, i - j >= 2l  (merged strided, beyond band)
+  RULE_SUMMARY = 5,         // j mod l >= l - c                 (fixed A2)
+  RULE_SUMMARY_EARLIER = 6  // j mod l >= l - c, floor(j/l) < floor(i/l) (merged fixed)
+};
+
+enum TileFlag : uint8_t { TILE_FULL = 0, TILE_PARTIAL = 1 };
+
+// ---- device-side schedule records (plain old data, copied as is) ----------
+
+// Forward work item: one query tile of one head class, with its key tiles.
+struct FwdItem {
+  int32_t qtile;      // tile index in the query view
+  int32_t kbeg, kend; // range in the key-entry array
+  uint8_t hclass;     // head class (split: 0 even heads, 1 odd heads)
+  uint8_t qview;      // View
+  uint8_t merge;      // 1: merge with the O/LSE already in the outputs
+  uint8_t pad;
+};
+
+struct KeyEnt {
+  int32_t ktile;  // tile index in the key view
+  uint8_t kview;  // View
+  uint8_t rule;   // Rule
+  uint8_t flag;   // TileFlag
+  uint8_t pad;
+};
+
+// Backward work item: one key tile of one segment, with its query tiles.
+struct BwdItem {
+  int32_t ktile;
+  int32_t qbeg, qend;  // range in the query-entry array
+  uint8_t hclass;
+  uint8_t kview;
+  uint8_t qview;
+  uint8_t rule;
+};
+
+struct QEnt {
+  int32_t qtile;
+  uint8_t flag;
+  uint8_t pad[3];
+};
+
+// Geometry every kernel needs to map view rows to natural positions.
+struct Geom {
+  int32_t T, l, c;
+  int32_t P;       // rows per residue class, T / l (0 when no class view)
+  int32_t ptiles;  // 128-row tiles per class, ceil(P / 128)
+  int32_t nsum;    // packed summary rows, (T / l) * c (0 when no summary view)
+  int32_t kind, mode;
+};
+
+// ---- host-side layout ------------------------------------------------------
+
+struct Tile {
+  int32_t q, k, live;
+  uint8_t flag;
+};
+
+struct Segment {
+  uint8_t qview, kview, rule;
+  int32_t nq, nk;            // tiles in the query / key view
+  std::vector<Tile> tiles;   // sorted by (q, k)
+};
+
+struct HeadClass {
+  std::vector<Segment> segs;
+  int64_t nnz = 0;
+};
+
+struct DeviceSchedule {
+  void* fwd_items[2] = {nullptr, nullptr};  // per forward pass
+  int32_t n_fwd_items[2] = {0, 0};
+  void* key_ents = nullptr;
+  void* bwd_items = nullptr;
+  int32_t n_bwd_items = 0;
+  void* q_ents = nullptr;
+  int32_t max_fwd_keys = 0;    // longest key list of a forward item
+};
+
+}  // namespace st
+
+struct st_layout {
+  st_pattern_desc desc;
+  st::Geom geom;
+  std::vector<st::HeadClass> hcs;
+  int32_t n_passes = 1;      // forward passes (2 for merged strided with class view)
+  bool tc_ok = false;        // every segment's rows are intervals (tensor-core path usable)
+  // host copies of the schedule
+  std::vector<st::FwdItem> fwd_items[2];
+  std::vector<st::KeyEnt> key_ents;
+  std::vector<st::BwdItem> bwd_items;
+  std::vector<st::QEnt> q_ents;
+  bool on_device = false;
+  int device = -1;
+  st::DeviceSchedule dev;
+};
+
+namespace st {
+// Implemented in layout.cpp.
+st_status build_layout(const st_pattern_desc* desc, st_layout* L);
+// Natural-order tiling of the whole set of a head class (export only).
+void natural_tiles(const st_layout* L, int hc, std::vector<Tile>& out);
+}  // namespace st

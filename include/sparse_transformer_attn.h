@@ -1,0 +1,195 @@
+/*
+ * sparse_transformer_attn.h - C ABI of libsparse_transformer_attn.so
+ *
+ * Causal self-attention restricted to the factorized patterns of the Sparse
+ * Transformer, forward and backward, as block-sparse attention on NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation ("Sparse Transformer" milestone page, nlp-lineage, "The idea",
+ * paragraph "The notation"): for every head and query position i,
+ *     O_i = softmax(q_i K_{S_i}^T * scale) V_{S_i},   scale = 1/sqrt(d),
+ * where S_i is the head's allowed key set; the softmax normalises over S_i
+ * only ("Sparse Transformer", llm-arch-kb, section 2 Derivation, "Sparse
+ * attention as an unnormalized form"). Positions are 0-indexed.
+ *   strided ("Pattern A"): A1_i = { j : max(0, i-l) <= j <= i }
+ *                           A2_i = { j <= i : (i-j) mod l == 0 }
+ *   fixed   ("Pattern B"): A1_i = { j <= i : floor(j/l) == floor(i/l) }
+ *                           A2_i = { j <= i : j mod l >= l-c }
+ *   dense causal:          S_i  = { j <= i }   (the comparator)
+ * Heads: split  - head h uses A1 when h is even, A2 when h is odd
+ *                 (milestone page, "The idea": each pattern is split between
+ *                 two heads);
+ *        merged - every head uses A1 u A2.
+ * The backward pass recomputes the attention matrix from the saved
+ * log-sum-exp instead of storing it (milestone page, "The idea",
+ * "Recomputation").
+ *
+ * Conventions for every call below:
+ *  - Tensors are caller-owned device pointers, contiguous [B, H, T, d]
+ *    row-major, 16-byte aligned, all of one dtype (st_dtype). LSE is float32
+ *    [B, H, T], natural log. The library owns only st_layout objects.
+ *  - fwd and bwd enqueue work on `stream` (a cudaStream_t passed as void*;
+ *    NULL = legacy default stream); they never allocate, never synchronise,
+ *    and return as soon as the work is queued.
+ *  - scale <= 0 selects 1/sqrt(d).
+ *  - Errors are returned as st_status; nothing is thrown across the ABI.
+ *    Invalid arguments return ST_ERR_INVALID before any launch; shapes the
+ *    kernels do not implement return ST_ERR_UNSUPPORTED before any launch.
+ *  - Supported shapes: bf16 with d = 64 (tensor-core path), float32 with
+ *    d = 32 or 64 (exact fp32 path). T must be a multiple of 128; l must
+ *    divide T or be >= T; for the fixed pattern with l < T, c must divide 128
+ *    and satisfy 1 <= c <= l.
+ */
+#ifndef SPARSE_TRANSFORMER_ATTN_H
+#define SPARSE_TRANSFORMER_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ST_OK = 0,
+  ST_ERR_INVALID = 1,        /* bad argument: null pointer, bad size, mismatch */
+  ST_ERR_UNSUPPORTED = 2,    /* valid, but not implemented by these kernels    */
+  ST_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed              */
+  ST_ERR_DEVICE_TIMEOUT = 4, /* a bounded on-device wait ran out               */
+  ST_ERR_WORKSPACE = 5       /* workspace missing or too small                 */
+} st_status;
+
+typedef enum { ST_STRIDED = 0, ST_FIXED = 1, ST_DENSE_CAUSAL = 2 } st_pattern_kind;
+typedef enum { ST_HEADS_SPLIT = 0, ST_HEADS_MERGED = 1 } st_head_mode;
+typedef enum { ST_F32 = 0, ST_BF16 = 1 } st_dtype;
+
+/* Pattern of one attention layer. l is the stride / block length
+ * ("Sparse Transformer", llm-arch-kb, section 2: l ~ sqrt(T)); c is the number
+ * of summary positions per block (fixed pattern only, 1 <= c <= l; ignored
+ * otherwise). head_mode is ignored for ST_DENSE_CAUSAL. */
+typedef struct {
+  int32_t kind;      /* st_pattern_kind */
+  int32_t head_mode; /* st_head_mode    */
+  int32_t T;
+  int32_t l;
+  int32_t c;
+} st_pattern_desc;
+
+/* Opaque, library-owned block layout of one pattern (host copy plus device
+ * copy). */
+typedef struct st_layout st_layout;
+
+/* Builds the block layout of a pattern ("Sparse Transformer", llm-arch-kb,
+ * section 3: the per-query key indices are precomputed and the attention is a
+ * block-sparse matmul). Every head's set S_i is split into disjoint segments;
+ * each segment lists, per 128-query tile, its live 128-key tiles (CSR) and,
+ * per key tile, its live query tiles (CSC), with a FULL/PARTIAL flag and the
+ * live-pair count of every tile. Segments read keys in natural order, in
+ * summary order (the last c positions of every block, packed) or in residue
+ * order (positions p*l + r of one class r), so that their tiles are dense.
+ * The device copy is uploaded with cudaMemcpyAsync on `stream`; the call
+ * synchronises that stream once before returning. Runs once per shape.
+ * Returns ST_ERR_INVALID for T < 1, l < 1, c outside [1, l] (fixed), or an
+ * unknown kind/mode; ST_ERR_CUDA if the upload fails (no layout returned). */
+st_status st_pattern_layout(const st_pattern_desc* desc, st_layout** out, void* stream);
+
+/* Same, host copy only (no CUDA call; usable without a GPU, e.g. to inspect
+ * or export a layout). fwd/bwd reject a host-only layout with
+ * ST_ERR_INVALID. */
+st_status st_pattern_layout_host(const st_pattern_desc* desc, st_layout** out);
+
+void st_layout_destroy(st_layout* layout);
+
+/* Numbers of head classes (2 for split heads: even, odd; else 1) and of
+ * segments per head class. */
+st_status st_layout_counts(const st_layout* layout, int32_t* n_head_classes,
+                           int32_t* n_segments);
+
+/* Key/query views and the membership rule of one segment:
+ * view 0 natural, 1 summary (keys only), 2 residue class. */
+st_status st_layout_segment_info(const st_layout* layout, int32_t head_class, int32_t segment,
+                                 int32_t* query_view, int32_t* key_view, int32_t* rule);
+
+/* Exports one segment's tile lists, or with segment = -1 the plain
+ * natural-order 128x128 tiling of the whole set S_{h,i} of the head class.
+ * transpose = 0 gives CSR over query tiles (ptr has n_query_tiles+1 entries,
+ * idx = key tile), transpose = 1 gives CSC over key tiles. Tiles are listed in
+ * ascending index order. flags[t] = 0 FULL (all 128x128 pairs live), 1
+ * PARTIAL; live[t] = number of live pairs. sizes_inout[0] / [1] give the
+ * capacities of ptr and of idx/flags/live; on return they hold the sizes
+ * needed. Any output pointer may be NULL (size query). Returns ST_ERR_INVALID
+ * for a bad head class or segment, ST_ERR_WORKSPACE if a capacity is short
+ * (sizes are still written). */
+st_status st_layout_export(const st_layout* layout, int32_t head_class, int32_t segment,
+                           int32_t transpose, int32_t* ptr, int32_t* idx, uint8_t* flags,
+                           int32_t* live, int64_t* sizes_inout);
+
+/* Live pairs of one head of the class (sum over i of |S_i|). */
+st_status st_layout_nnz(const st_layout* layout, int32_t head_class, int64_t* nnz);
+
+/* Forward: O and LSE for all B*H heads. Head h = index within H of the
+ * [B, H, T, d] tensors (split mode picks A1/A2 from its parity). Rows with an
+ * empty set get O = 0 and LSE = -inf. For a strided merged layout the call
+ * runs two passes (natural-order window keys, then residue-order strided
+ * keys) and merges them by log-sum-exp in place in o and lse. */
+st_status st_sparse_attn_fwd(const st_layout* layout, st_dtype dtype, int32_t B, int32_t H,
+                             int32_t T, int32_t d, float scale, const void* q, const void* k,
+                             const void* v, void* o, float* lse, void* stream);
+
+/* Bytes of device workspace st_sparse_attn_bwd needs for these sizes. */
+st_status st_sparse_attn_bwd_workspace(const st_layout* layout, st_dtype dtype, int32_t B,
+                                       int32_t H, int32_t T, int32_t d, size_t* bytes);
+
+/* Backward: dQ, dK, dV (dtype of the inputs, fp32 accumulation) from Q, K,
+ * V, the forward's O and LSE, and the upstream gradient dout. P is recomputed
+ * as exp(s - LSE) on live tiles; D_i = dout_i . O_i. The workspace (device
+ * memory, at least st_sparse_attn_bwd_workspace bytes, 256-byte aligned) is
+ * overwritten; it holds the fp32 accumulators and D. Returns
+ * ST_ERR_WORKSPACE if it is missing or too small. */
+st_status st_sparse_attn_bwd(const st_layout* layout, st_dtype dtype, int32_t B, int32_t H,
+                             int32_t T, int32_t d, float scale, const void* q, const void* k,
+                             const void* v, const void* o, const float* lse, const void* dout,
+                             void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                             void* stream);
+
+/* Synchronises `stream`, then returns and clears the device-side status word
+ * that the kernels set when a bounded wait runs out (ST_ERR_DEVICE_TIMEOUT) or
+ * an index check fails (ST_ERR_INVALID); ST_ERR_CUDA if the sync fails. */
+st_status st_last_device_status(void* stream);
+
+/* Upper bound, in nanoseconds, of every on-device wait of later launches
+ * (default 2e9). 0 restores the default. A wait that runs out sets the status
+ * word and makes the kernel return early. For tests of the timeout path only,
+ * force_timeout != 0 makes the next forward launch skip the loads of its
+ * first key tile so its waits run out on purpose (the GPU stays usable). */
+st_status st_set_wait_limit(uint64_t ns, int32_t force_timeout);
+
+/* Kernel launches one fwd / bwd call makes with this layout and dtype (the
+ * forward runs one launch per pass; the backward a prologue, its main
+ * kernel(s) and, for bf16, an epilogue). */
+st_status st_layout_launches(const st_layout* layout, st_dtype dtype, int32_t* fwd_launches,
+                             int32_t* bwd_launches);
+
+/* Benchmark instrumentation. enable != 0 creates (once) two pairs of CUDA
+ * events on the current device; from then on every fwd call records pair 0
+ * around its attention launches and every bwd call records pair 1 around its
+ * main attention kernel, on the call's stream. enable = 0 stops recording.
+ * Events are created here, never inside fwd/bwd. */
+st_status st_kernel_timing(int32_t enable);
+
+/* Milliseconds between the pair of events of the latest call of `kernel`
+ * (0 = forward attention launches, 1 = backward main kernel); synchronises on
+ * that call's stop event. ST_ERR_INVALID if timing is off or nothing ran. */
+st_status st_kernel_elapsed_ms(int32_t kernel, float* ms);
+
+/* Static description of a status code. */
+const char* st_status_string(st_status status);
+
+/* Library version, "major.minor.patch". */
+const char* st_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_TRANSFORMER_ATTN_H */

@@ -1,0 +1,156 @@
+"""GPU parity: the CUDA path (through the C ABI) vs the oracle, element by
+element on the same seeded inputs, at sizes that span several tiles and
+ragged tails; then sampled rows at the full workload sizes."""
+import numpy as np
+import pytest
+import torch
+
+import factorized_sparse_self_b200 as st
+import synth
+from gpu_util import compare, compare_lse, device_inputs, f32, run_library
+
+pytestmark = pytest.mark.gpu
+
+# kind, mode, B, H, T, d, l, c, dtype, std
+SMALL = [
+    # the fp32 workload itself (strided split, T = 256, d = 32, l = 16)
+    ("strided", "split", 1, 2, 256, 32, 16, 1, "f32", 1.0),
+    ("fixed", "merged", 1, 2, 384, 64, 48, 6, "f32", 1.0),
+    ("strided", "merged", 2, 2, 300, 32, 20, 1, "f32", 1.0),  # ragged T, no class view
+    # bf16 tensor-core path
+    ("fixed", "split", 1, 4, 1024, 64, 64, 8, "bf16", 64 ** -0.25),
+    ("fixed", "merged", 1, 2, 1536, 64, 128, 8, "bf16", 0.5),
+    ("fixed", "merged", 2, 2, 1024, 64, 32, 1, "bf16", 0.5),
+    ("fixed", "split", 1, 2, 768, 64, 96, 32, "bf16", 0.5),
+    ("strided", "split", 1, 4, 1536, 64, 192, 1, "bf16", 0.5),   # 8-row residue classes
+    ("strided", "merged", 1, 2, 2048, 64, 256, 1, "bf16", 0.5),
+    ("strided", "split", 1, 2, 1024, 64, 16, 1, "bf16", 0.5),    # 64-row classes, l << 128
+    ("strided", "merged", 1, 2, 512, 64, 8, 1, "bf16", 0.5),
+    ("dense", "merged", 1, 2, 640, 64, 1, 1, "bf16", 0.5),
+    ("strided", "merged", 1, 2, 256, 64, 300, 1, "bf16", 0.5),   # l > T: full causal
+    ("strided", "split", 1, 2, 384, 64, 384, 1, "bf16", 0.5),    # l = T: A2 is the diagonal
+    ("fixed", "split", 1, 2, 256, 64, 300, 8, "bf16", 0.5),      # l > T
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "-".join(map(str, c[:8])) + "-" + c[8])
+def test_parity_small(orc, case):
+    kind, mode, B, H, T, d, l, c, dtype, std = case
+    (q, k, v, do), (qd, kd, vd, dod) = device_inputs(B, H, T, d, dtype, std, seed=0)
+    L = st.st_pattern_layout(kind, mode, T, l, c)
+    o, lse, (dq, dk, dv) = run_library(L, qd, kd, vd, dod)
+    ro, rlse = orc.forward(kind, mode, f32(q), f32(k), f32(v), l, c)
+    rdq, rdk, rdv = orc.backward(kind, mode, f32(q), f32(k), f32(v), f32(do), l, c)
+    tag = str(case)
+    compare("O", f32(o.cpu()), ro, dtype, tag)
+    compare_lse(lse.cpu().numpy(), rlse, dtype, tag)
+    compare("dQ", f32(dq.cpu()), rdq, dtype, tag)
+    compare("dK", f32(dk.cpu()), rdk, dtype, tag)
+    compare("dV", f32(dv.cpu()), rdv, dtype, tag)
+
+
+@pytest.mark.parametrize("name", [n for n in synth.ORDER if synth.WORKLOADS[n].dtype == "bf16"])
+def test_parity_full_size_sampled(orc, name):
+    """Full workload sizes, launched as the benchmark launches them: sampled
+    output rows vs the oracle row by row (forward rows, dQ rows, dK / dV rows)."""
+    w = synth.WORKLOADS[name]
+    (q, k, v, do), (qd, kd, vd, dod) = device_inputs(w.B, w.H, w.T, w.d, w.dtype, w.std, seed=0)
+    L = st.st_pattern_layout(w.kind, w.mode, w.T, w.l, w.c)
+    o, lse, (dq, dk, dv) = run_library(L, qd, kd, vd, dod)
+    rng = np.random.default_rng(1)
+    BH = w.B * w.H
+    n = 24
+    bh = rng.integers(0, BH, n)
+    rows = np.concatenate([rng.integers(0, w.T, n - 4), [0, w.T - 1, w.l - 1, w.l]])
+    # include the last summary key of block 0 and the first row of block 1
+    qf, kf, vf, dof = f32(q), f32(k), f32(v), f32(do)
+    ro, rlse = orc.forward_rows(w.kind, w.mode, qf, kf, vf, w.l, w.c, bh, rows)
+    go = f32(o.cpu()).reshape(BH, w.T, w.d)[bh, rows]
+    compare("O rows", go, ro, "bf16", name)
+    compare_lse(lse.cpu().numpy().reshape(BH, w.T)[bh, rows], rlse, "bf16", name)
+    rdq = orc.backward_query_rows(w.kind, w.mode, qf, kf, vf, dof, w.l, w.c, bh, rows)
+    compare("dQ rows", f32(dq.cpu()).reshape(BH, w.T, w.d)[bh, rows], rdq, "bf16", name)
+    nk = 6
+    kb, kr = bh[:nk], rows[:nk].copy()
+    if w.kind == "fixed":
+        kr[0] = w.l - 1  # a summary key, attended by every later block
+    rdk, rdv = orc.backward_key_rows(w.kind, w.mode, qf, kf, vf, dof, w.l, w.c, kb, kr)
+    compare("dK rows", f32(dk.cpu()).reshape(BH, w.T, w.d)[kb, kr], rdk, "bf16", name)
+    compare("dV rows", f32(dv.cpu()).reshape(BH, w.T, w.d)[kb, kr], rdv, "bf16", name)
+
+
+def test_full_size_invariants():
+    """At the largest text-like size: every output finite, empty rows absent,
+    LSE >= max over the diagonal logit, and rows of dK sum to ~0 per head."""
+    w = synth.WORKLOADS["fixed-merged-T12288"]
+    (_, _, _, _), (qd, kd, vd, dod) = device_inputs(w.B, w.H, w.T, w.d, w.dtype, w.std)
+    L = st.st_pattern_layout(w.kind, w.mode, w.T, w.l, w.c)
+    o, lse, (dq, dk, dv) = run_library(L, qd, kd, vd, dod)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    sii = (qd.float() * kd.float()).sum(-1) / 8.0
+    assert (lse >= sii - 1e-2).all()
+    s = dk.float().sum(dim=2)
+    assert s.abs().max().item() < 0.05 * dk.float().abs().sum(dim=2).max().item()
+
+
+def test_forward_is_deterministic_and_guard_regions_untouched():
+    w = synth.WORKLOADS["strided-split-T12288"]
+    B, H, T, d = 1, 4, w.T, w.d
+    (_, _, _, _), (qd, kd, vd, dod) = device_inputs(B, H, T, d, "bf16", 0.5)
+    L = st.st_pattern_layout(w.kind, w.mode, T, w.l, w.c)
+    pad = 4096
+    buf = torch.full((B * H * T * d + 2 * pad,), 7.0, dtype=torch.bfloat16, device="cuda")
+    o = buf[pad:pad + B * H * T * d].view(B, H, T, d)
+    lbuf = torch.full((B * H * T + 2 * pad,), 3.0, dtype=torch.float32, device="cuda")
+    lse = lbuf[pad:pad + B * H * T].view(B, H, T)
+    st.st_sparse_attn_fwd(L, qd, kd, vd, o=o, lse=lse)
+    o1, l1 = o.clone(), lse.clone()
+    st.st_sparse_attn_fwd(L, qd, kd, vd, o=o, lse=lse)
+    torch.cuda.synchronize()
+    assert st.st_last_device_status() == st.ST_OK
+    assert torch.equal(o, o1) and torch.equal(lse, l1)
+    assert (buf[:pad] == 7.0).all() and (buf[-pad:] == 7.0).all()
+    assert (lbuf[:pad] == 3.0).all() and (lbuf[-pad:] == 3.0).all()
+
+
+def test_bad_arguments_rejected_before_launch():
+    L = st.st_pattern_layout("fixed", "split", 1024, 64, 8)
+    q = torch.zeros(1, 2, 1024, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(st.StatusError) as e:
+        st.st_sparse_attn_fwd(L, q[:, :, :512].contiguous(), q[:, :, :512].contiguous(),
+                              q[:, :, :512].contiguous())
+    assert e.value.code == st.ST_ERR_INVALID
+    q32 = torch.zeros(1, 2, 1024, 32, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(st.StatusError) as e:
+        st.st_sparse_attn_fwd(L, q32, q32, q32)
+    assert e.value.code == st.ST_ERR_UNSUPPORTED
+    o = torch.empty_like(q)
+    lse = torch.empty(1, 2, 1024, device="cuda")
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(st.StatusError) as e:
+        st.st_sparse_attn_bwd(L, q, q, q, o, lse, q, workspace=ws)
+    assert e.value.code == st.ST_ERR_WORKSPACE
+    Lr = st.st_pattern_layout("strided", "merged", 1000, 48, 1)
+    qr = torch.zeros(1, 2, 1000, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(st.StatusError) as e:
+        st.st_sparse_attn_fwd(Lr, qr, qr, qr)
+    assert e.value.code == st.ST_ERR_UNSUPPORTED
+
+
+def test_device_wait_timeout_reports_and_recovers(orc):
+    """A forward launch whose first key-tile load is skipped on purpose: its
+    bounded waits run out, the status word reports the timeout, and the next
+    normal call on the same context is correct."""
+    kind, mode, B, H, T, d, l, c = "fixed", "merged", 1, 2, 1024, 64, 128, 8
+    (q, k, v, do), (qd, kd, vd, dod) = device_inputs(B, H, T, d, "bf16", 0.5)
+    L = st.st_pattern_layout(kind, mode, T, l, c)
+    st.st_set_wait_limit(20_000_000, force_timeout=True)
+    try:
+        st.st_sparse_attn_fwd(L, qd, kd, vd)
+        assert st.st_last_device_status() == st.ST_ERR_DEVICE_TIMEOUT
+    finally:
+        st.st_set_wait_limit(0, force_timeout=False)
+    assert st.st_last_device_status() == st.ST_OK
+    o, lse, _ = run_library(L, qd, kd, vd, dod, backward=False)
+    ro, rlse = orc.forward(kind, mode, f32(q), f32(k), f32(v), l, c)
+    compare("O", f32(o.cpu()), ro, "bf16")

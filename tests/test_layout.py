@@ -1,0 +1,92 @@
+"""Host layout builder vs the oracle's re-derivation from the explicit sets.
+
+The library computes tiles from closed-form row intervals; the oracle walks
+every live (i, j) pair. They must agree bit for bit: the same segments and
+views, the same tiles in the same order, the same live counts and flags.
+Runs on the CPU (host-only layouts, no CUDA call)."""
+import numpy as np
+import pytest
+
+import factorized_sparse_self_b200 as st
+
+CASES = [
+    # kind, mode, T, l, c
+    ("fixed", "split", 1024, 64, 8),
+    ("fixed", "merged", 1536, 128, 8),
+    ("fixed", "split", 768, 96, 4),
+    ("fixed", "merged", 512, 64, 64),
+    ("fixed", "merged", 640, 40, 5),        # c does not divide 128: natural-order summary keys
+    ("fixed", "split", 384, 48, 16),
+    ("strided", "split", 1536, 192, 1),
+    ("strided", "merged", 2048, 256, 1),
+    ("strided", "split", 1024, 16, 1),
+    ("strided", "merged", 1024, 32, 1),
+    ("strided", "merged", 1000, 48, 1),     # T not a multiple of l: no class view
+    ("strided", "split", 384, 384, 1),      # l = T
+    ("strided", "merged", 256, 1000, 1),    # l > T
+    ("fixed", "split", 256, 300, 7),        # l > T
+    ("dense", "merged", 640, 1, 1),
+    ("dense", "merged", 200, 1, 1),         # ragged T
+]
+
+
+def _triples(ptr, idx, live, transpose):
+    rows = np.repeat(np.arange(len(ptr) - 1), np.diff(ptr))
+    if transpose:
+        return idx.astype(np.int64), rows.astype(np.int64), live.astype(np.int64)
+    return rows.astype(np.int64), idx.astype(np.int64), live.astype(np.int64)
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_layout_bit_exact_vs_oracle(orc, case):
+    kind, mode, T, l, c = case
+    L = st.st_pattern_layout_host(kind, mode, T, l, c)
+    nhc, nseg = L.counts()
+    assert nhc == orc.num_head_classes(kind, mode)
+    assert nseg == orc.num_segments(kind, mode)
+    for hc in range(nhc):
+        total = 0
+        for seg in list(range(nseg)) + [-1]:
+            if seg >= 0:
+                qv, kv, _ = L.segment_info(hc, seg)
+                assert (qv, kv) == orc.segment_views(kind, mode, T, l, c, hc, seg)
+            oq, ok, olive = orc.layout_tiles(kind, mode, T, l, c, hc, seg)
+            ptr, idx, flags, live = L.export(hc, seg, transpose=False)
+            q, k, lv = _triples(ptr, idx, live, False)
+            np.testing.assert_array_equal(q, oq)
+            np.testing.assert_array_equal(k, ok)
+            np.testing.assert_array_equal(lv, olive)
+            np.testing.assert_array_equal(flags, (olive != 128 * 128).astype(np.uint8))
+            # the CSC export lists the same tiles, key-major
+            ptr_t, idx_t, flags_t, live_t = L.export(hc, seg, transpose=True)
+            q2, k2, lv2 = _triples(ptr_t, idx_t, live_t, True)
+            order = np.lexsort((oq, ok))
+            np.testing.assert_array_equal(q2, oq[order])
+            np.testing.assert_array_equal(k2, ok[order])
+            np.testing.assert_array_equal(lv2, olive[order])
+            if seg >= 0:
+                total += int(live.sum())
+        h = hc if mode == "split" else 0
+        assert total == L.nnz(hc) == orc.nnz(kind, mode, T, l, c, h)
+
+
+def test_gathered_views_make_tiles_dense(orc):
+    """The gather views are what make the live tiles dense: tile efficiency of
+    the segment tilings vs the plain natural tiling, text-like fixed pattern."""
+    L = st.st_pattern_layout_host("fixed", "merged", 12288, 128, 8)
+    live_seg = sum(int(L.export(0, s)[3].sum()) for s in range(2))
+    area_seg = sum(len(L.export(0, s)[1]) for s in range(2)) * 128 * 128
+    _, idx, _, live_nat = L.export(0, -1)
+    eff_seg = live_seg / area_seg
+    eff_nat = live_nat.sum() / (len(idx) * 128 * 128)
+    assert live_seg == live_nat.sum() == 5462016
+    assert eff_seg > 0.75 and eff_nat < 0.08
+
+
+def test_invalid_descriptors_rejected():
+    for args in [("fixed", "split", 256, 16, 0), ("fixed", "split", 256, 16, 17),
+                 ("strided", "split", 256, 0, 1), ("strided", "split", 0, 4, 1),
+                 (7, "split", 256, 16, 1), ("strided", 5, 256, 16, 1)]:
+        with pytest.raises(st.StatusError) as e:
+            st.st_pattern_layout_host(*args)
+        assert e.value.code == st.ST_ERR_INVALID
