@@ -43,6 +43,9 @@ SIGNATURES = {
     "st_sparse_attn_bwd": (ctypes.c_int, [_P, ctypes.c_int, _i32, _i32, _i32, _i32,
                                           ctypes.c_float, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                           _P, ctypes.c_size_t, _P]),
+    "st_sparse_attn_bwd_noalloc": (ctypes.c_int, [_P, ctypes.c_int, _i32, _i32, _i32, _i32,
+                                                  ctypes.c_float, _P, _P, _P, _P, _P, _P, _P, _P,
+                                                  _P, _P]),
     "st_last_device_status": (ctypes.c_int, [_P]),
     "st_set_wait_limit": (ctypes.c_int, [_u64, _i32]),
     "st_layout_launches": (ctypes.c_int, [_P, ctypes.c_int, _P, _P]),
@@ -233,6 +236,24 @@ def st_sparse_attn_bwd(layout: Layout, q, k, v, o, lse, dout, scale=None, worksp
                                     ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
                                     _stream_ptr(stream))
     _check(code, "st_sparse_attn_bwd")
+    return dq, dk, dv
+
+
+def st_sparse_attn_bwd_noalloc(layout: Layout, q, k, v, o, lse, dout, dq, dk, dv, scale=None,
+                               stream=None):
+    """Backward for callers that cannot allocate device memory: same result as
+    st_sparse_attn_bwd, with the scratch in a fixed 64 MiB library-owned
+    device array instead of a caller workspace. The caller passes every output
+    buffer; nothing is allocated here or in the library. Calls whose GPU work
+    overlaps share that array and race, so serialise them."""
+    B, H, T, d = q.shape
+    ptrs = [_need(x, n, q) for x, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"),
+                                        (dq, "dq"), (dk, "dk"), (dv, "dv"))]
+    code = lib().st_sparse_attn_bwd_noalloc(layout.handle, _dtype_code(q), B, H, T, d,
+                                            float(scale) if scale else 0.0, ptrs[0], ptrs[1],
+                                            ptrs[2], ptrs[3], _need(lse, "lse"), ptrs[4], ptrs[5],
+                                            ptrs[6], ptrs[7], _stream_ptr(stream))
+    _check(code, "st_sparse_attn_bwd_noalloc")
     return dq, dk, dv
 
 

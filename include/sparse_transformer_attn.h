@@ -152,6 +152,31 @@ st_status st_sparse_attn_bwd(const st_layout* layout, st_dtype dtype, int32_t B,
                              void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                              void* stream);
 
+/* Backward pass for callers that cannot allocate device memory. The paper
+ * has no counterpart: this is a deployment convenience of this library.
+ * Some callers cannot call cudaMalloc or keep a workspace between calls
+ * (a plugin whose host application owns every device allocation, or a
+ * latency-critical path that must not allocate). This entry point computes
+ * exactly what st_sparse_attn_bwd computes, with the same arguments except
+ * the workspace: its scratch is a fixed 64 MiB array of library-owned device
+ * memory that every GPU which loads the library holds until the process
+ * exits. It never allocates.
+ *  - Limit: st_sparse_attn_bwd_workspace bytes for these sizes must not
+ *    exceed 64 MiB (bf16: B*H*T*(4 + 12*d) bytes, rounded up); larger
+ *    calls return ST_ERR_WORKSPACE before any launch.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the one array, and it keeps the last call's
+ *    contents (each call re-zeroes what must start at zero). Calls whose GPU
+ *    work overlaps (other streams, other host threads) race on it and give
+ *    wrong gradients: serialise them. */
+st_status st_sparse_attn_bwd_noalloc(const st_layout* layout, st_dtype dtype, int32_t B, int32_t H,
+                                     int32_t T, int32_t d, float scale, const void* q,
+                                     const void* k, const void* v, const void* o,
+                                     const float* lse, const void* dout, void* dq, void* dk,
+                                     void* dv, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device-side status word
  * that the kernels set when a bounded wait runs out (ST_ERR_DEVICE_TIMEOUT) or
  * an index check fails (ST_ERR_INVALID); ST_ERR_CUDA if the sync fails. */
