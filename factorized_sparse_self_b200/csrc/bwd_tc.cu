@@ -10,17 +10,24 @@
 //   dV  += P^T dO                 (M=128, N=64, K=128)
 //   dK  += dS^T Q
 //   dQ_i = dS K  -> TMA reduce-add into the fp32 dQ accumulator
-// dV and dK stay in TMEM for the whole key tile and are reduced into fp32
-// accumulators at the end (a key tile can belong to two segments of a merged
-// head); an epilogue kernel applies the scale and rounds to bf16.
+// dV and dK stay in TMEM for a whole work unit (a key tile, or a chunk of a
+// long key column) and are reduce-added into fp32 accumulators at its end; an
+// epilogue kernel applies the scale and rounds to bf16.
 //
-// Warp roles: warp 0 TMA producer (K, V once; Q, dO per query tile into a
-// 2-stage ring, with LSE and D by plain loads); warp 1 TMEM owner and MMA
-// issuer; warps 2..5 compute (thread = key row = TMEM lane for S^T / dP^T,
-// and query row for draining dQ). The MMA warp issues S, dP of the next tile
-// before dV, dK, dQ of the current one, so the exponentials overlap the
-// tensor pipe. All waits are bounded.
+// Persistent CTAs, one per SM, each walking a strided share of the work units
+// (longest first). Warpgroup roles:
+//   warpgroups 0, 1  compute: thread = key row = TMEM lane for S^T / dP^T;
+//                    warpgroup w owns query columns 64w .. 64w+63 of every
+//                    tile, the dQ columns 32w .. 32w+31, and drains dK (w = 0)
+//                    or dV (w = 1) at the end of a unit;
+//   warpgroup 2      warp 8 TMA producer (K, V per unit; Q, dO per query
+//                    tile into a 2-stage ring, with LSE and D by plain loads),
+//                    warp 9 TMEM owner and MMA issuer.
+// The MMA warp issues S, dP of the next tile before dV, dK, dQ of the current
+// one, so the exponentials overlap the tensor pipe. All waits are bounded.
 #include <math.h>
+
+#include <algorithm>
 
 #include "launch.h"
 #include "tc_common.cuh"
@@ -32,7 +39,9 @@ using namespace tc;
 
 constexpr int NS = 2;
 constexpr int kTileBytes = kTile * 64 * 2;  // 128 x 64 bf16 = 16 KB
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
+constexpr uint32_t kRegsCompute = 208, kRegsIssue = 88;  // launch: 168 per thread
+static_assert(256 * kRegsCompute + 128 * kRegsIssue == kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -52,9 +61,9 @@ struct SmemBwd {
   uint8_t stage[2 * kTileBytes]; // fp32 dQ tile for the reduce: two 32-column halves
   float l2[NS][kTile];           // LSE_i * log2(e) of the stage's query rows
   float dd[NS][kTile];           // D_i
-  uint64_t kv_full, full[NS], empty[NS];
+  uint64_t kv_full, kv_done, full[NS], empty[NS];
   uint64_t s_full, dp_full, ds_ready, pds_free, dq_full, dq_free, stg_full, stg_free;
-  uint64_t kv_done, out_full, fin;
+  uint64_t acc_free, out_full, kvstg_free, fin;
   uint32_t tmem_base;
   int abort;
 };
@@ -127,42 +136,53 @@ __device__ __forceinline__ void live_rows(const Geom& g, int kview, int qview, i
   if (hi < lo) hi = lo;
 }
 
+struct Unit {
+  BwdItem it;
+  int bh;
+};
+
+__device__ __forceinline__ Unit unit_of(const BwdItem* items, int u, int NH, int B, int H,
+                                        int nclasses) {
+  Unit x;
+  x.it = items[u / NH];
+  x.bh = head_of(u % NH, x.it.hclass, B, H, nclasses);
+  return x;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __restrict__ items,
-              const QEnt* __restrict__ qents, int B, int H, int nclasses, float scale_log2,
-              const float* __restrict__ lse, const float* __restrict__ Dg, int* status,
-              uint64_t wait_ns) {
+              int n_units, int NH, const QEnt* __restrict__ qents, int B, int H, int nclasses,
+              float scale_log2, const float* __restrict__ lse, const float* __restrict__ Dg,
+              int* status, uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   SmemBwd& S = *reinterpret_cast<SmemBwd*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
-  const BwdItem it = items[blockIdx.y];
-  const int bh = head_of(blockIdx.x, it.hclass, B, H, nclasses);
-  if (bh < 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n = it.qend - it.qbeg;
   volatile int* abort = &S.abort;
 
   if (threadIdx.x == 0) {
     mbar_init(&S.kv_full, 1);
+    mbar_init(&S.kv_done, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&S.full[s], 33);  // expect_tx arrive + 32 producer lanes
       mbar_init(&S.empty[s], 1);
     }
     mbar_init(&S.s_full, 1);
     mbar_init(&S.dp_full, 1);
-    mbar_init(&S.ds_ready, 128);
+    mbar_init(&S.ds_ready, 256);
     mbar_init(&S.pds_free, 1);
     mbar_init(&S.dq_full, 1);
-    mbar_init(&S.dq_free, 128);
-    mbar_init(&S.stg_full, 128);
+    mbar_init(&S.dq_free, 256);
+    mbar_init(&S.stg_full, 256);
     mbar_init(&S.stg_free, 1);
-    mbar_init(&S.kv_done, 1);
-    mbar_init(&S.out_full, 128);
+    mbar_init(&S.acc_free, 256);
+    mbar_init(&S.out_full, 256);
+    mbar_init(&S.kvstg_free, 1);
     mbar_init(&S.fin, 1);
     S.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 9) {
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -174,149 +194,188 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     set_status(status, ST_ERR_DEVICE_TIMEOUT);
   };
 
-  if (warp == 0) {
-    // ---------------- producer ----------------
-    int issued[NS] = {-1, -1};
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&S.kv_full, 2 * kTileBytes);
-      load_tile(S.k, maps.k, it.kview, g, it.ktile, bh, &S.kv_full);
-      load_tile(S.v, maps.v, it.kview, g, it.ktile, bh, &S.kv_full);
-    }
-    for (int e = 0; e < n; ++e) {
-      const int s = e % NS;
-      if (e >= NS) {
-        bool ok = mbar_wait(&S.empty[s], ((e / NS) - 1) & 1, wait_ns, abort);
-        if (!__all_sync(0xffffffffu, ok)) {
-          if (lane == 0) fail();
-          break;
+  if (warp >= 8) {
+    regs_decrease<kRegsIssue>();
+    if (warp == 8) {
+      // ---------------- producer ----------------
+      int full_last[NS] = {-1, -1};
+      int kv_last = -1;
+      bool ok = true;
+      int gt = 0, n = 0;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        const Unit x = unit_of(items, u, NH, B, H, nclasses);
+        if (x.bh < 0) continue;
+        const int cnt = x.it.qend - x.it.qbeg;
+        auto issue_q = [&](int e) -> bool {
+          const int s = gt % NS;
+          const bool w = mbar_wait(&S.empty[s], ((gt / NS) & 1) ^ 1, wait_ns, abort);
+          if (!__all_sync(0xffffffffu, w)) return false;
+          const QEnt qe = qents[x.it.qbeg + e];
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&S.full[s], 2 * kTileBytes);
+            load_tile(S.q[s], maps.q, x.it.qview, g, qe.qtile, x.bh, &S.full[s]);
+            load_tile(S.dout[s], maps.dout, x.it.qview, g, qe.qtile, x.bh, &S.full[s]);
+          }
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int row = lane + 32 * t;
+            const int i = view_pos(g, x.it.qview, qe.qtile, row);
+            // rows with an empty set (LSE = -inf) have no live pair; 0 keeps
+            // their masked exponents at -inf instead of -inf + inf
+            const float L = (i >= 0) ? lse[(size_t)x.bh * g.T + i] : 0.f;
+            S.l2[s][row] = (L > -INFINITY) ? L * kLog2e : 0.f;
+            S.dd[s][row] = (i >= 0) ? Dg[(size_t)x.bh * g.T + i] : 0.f;
+          }
+          mbar_arrive(&S.full[s]);
+          full_last[s] = gt;
+          ++gt;
+          return true;
+        };
+        // the first query tiles of the unit may load while the previous unit
+        // still holds the K / V buffers
+        const int pre = min(cnt, NS);
+        int e = 0;
+        for (; ok && e < pre; ++e) ok = issue_q(e);
+        if (!ok) break;
+        ok = __all_sync(0xffffffffu, mbar_wait(&S.kv_done, (n & 1) ^ 1, wait_ns, abort));
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&S.kv_full, 2 * kTileBytes);
+          load_tile(S.k, maps.k, x.it.kview, g, x.it.ktile, x.bh, &S.kv_full);
+          load_tile(S.v, maps.v, x.it.kview, g, x.it.ktile, x.bh, &S.kv_full);
         }
+        kv_last = n;
+        for (; ok && e < cnt; ++e) ok = issue_q(e);
+        ++n;
       }
-      const QEnt qe = qents[it.qbeg + e];
+      if (!ok && lane == 0) fail();
       if (lane == 0) {
-        mbar_arrive_expect_tx(&S.full[s], 2 * kTileBytes);
-        load_tile(S.q[s], maps.q, it.qview, g, qe.qtile, bh, &S.full[s]);
-        load_tile(S.dout[s], maps.dout, it.qview, g, qe.qtile, bh, &S.full[s]);
+        if (kv_last >= 0 && !mbar_wait(&S.kv_full, kv_last & 1, wait_ns, abort)) fail();
+        for (int s = 0; s < NS; ++s)
+          if (full_last[s] >= 0 &&
+              !mbar_wait(&S.full[s], (full_last[s] / NS) & 1, wait_ns, abort))
+            fail();
       }
+    } else if (warp == 9) {
+      // ---------------- MMA issuer ----------------
+      if (lane == 0) {
+        const uint32_t idSS = idesc_bf16(128, 128, false, false);
+        const uint32_t idKM = idesc_bf16(128, 64, false, true);  // A K-major, B MN-major
+        const uint32_t idMM = idesc_bf16(128, 64, true, true);   // A MN-major, B MN-major
+        const uint32_t k_addr = smem_u32(S.k), v_addr = smem_u32(S.v);
+        const uint32_t pt_addr = smem_u32(S.pt), ds_addr = smem_u32(S.dst);
+        bool ok = true;
+        int gt = 0, n = 0;
+        auto issue_s_dp = [&](int t) -> bool {
+          const int s = t % NS;
+          if (!mbar_wait(&S.full[s], (t / NS) & 1, wait_ns, abort)) return false;
+          tc_fence_after();
+          const uint32_t q_addr = smem_u32(S.q[s]), o_addr = smem_u32(S.dout[s]);
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const int row = lane + 32 * t;
-        const int i = view_pos(g, it.qview, qe.qtile, row);
-        S.l2[s][row] = (i >= 0) ? lse[(size_t)bh * g.T + i] * kLog2e : 0.f;
-        S.dd[s][row] = (i >= 0) ? Dg[(size_t)bh * g.T + i] : 0.f;
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + kColS, sdesc(k_addr + kk * 32, 16, 1024),
+                   sdesc(q_addr + kk * 32, 16, 1024), idSS, kk > 0);
+          mma_commit(&S.s_full);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + kColDP, sdesc(v_addr + kk * 32, 16, 1024),
+                   sdesc(o_addr + kk * 32, 16, 1024), idSS, kk > 0);
+          mma_commit(&S.dp_full);
+          return true;
+        };
+        for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+          const Unit x = unit_of(items, u, NH, B, H, nclasses);
+          if (x.bh < 0) continue;
+          const int cnt = x.it.qend - x.it.qbeg;
+          ok = mbar_wait(&S.kv_full, n & 1, wait_ns, abort);
+          if (ok) ok = issue_s_dp(gt);
+          for (int e = 0; ok && e < cnt; ++e, ++gt) {
+            const int s = gt % NS;
+            if (!mbar_wait(&S.ds_ready, gt & 1, wait_ns, abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (e + 1 < cnt && !issue_s_dp(gt + 1)) {
+              ok = false;
+              break;
+            }
+            if (e == 0 && !mbar_wait(&S.acc_free, (n & 1) ^ 1, wait_ns, abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t q_addr = smem_u32(S.q[s]), o_addr = smem_u32(S.dout[s]);
+            // dV += P^T dO ; dK += dS^T Q   (K = 128 queries, 8 steps of 16)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + kColDV,
+                     sdesc(pt_addr + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
+                     sdesc(o_addr + kk * 2048, 16384, 1024), idKM, (e > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + kColDK,
+                     sdesc(ds_addr + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
+                     sdesc(q_addr + kk * 2048, 16384, 1024), idKM, (e > 0 || kk > 0) ? 1u : 0u);
+            if (gt > 0 && !mbar_wait(&S.dq_free, (gt - 1) & 1, wait_ns, abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // dQ = dS K   (A = dS^T read MN-major, K = 128 keys)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + kColDQ, sdesc(ds_addr + kk * 2048, kTileBytes, 1024),
+                     sdesc(k_addr + kk * 2048, 16384, 1024), idMM, kk > 0 ? 1u : 0u);
+            mma_commit(&S.dq_full);
+            mma_commit(&S.pds_free);
+            mma_commit(&S.empty[s]);
+          }
+          if (!ok) break;
+          mma_commit(&S.kv_done);
+          ++n;
+        }
+        if (!ok) fail();
+        mma_commit(&S.fin);
+        mbar_wait(&S.fin, 0, wait_ns, abort);
       }
-      mbar_arrive(&S.full[s]);
-      issued[s] = e;
-    }
-    if (lane == 0) {
-      mbar_wait(&S.kv_full, 0, wait_ns, abort);
-      for (int s = 0; s < NS; ++s)
-        if (issued[s] >= 0 && !mbar_wait(&S.full[s], (issued[s] / NS) & 1, wait_ns, abort))
-          fail();
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      const uint32_t idSS = idesc_bf16(128, 128, false, false);
-      const uint32_t idKM = idesc_bf16(128, 64, false, true);  // A K-major, B MN-major
-      const uint32_t idMM = idesc_bf16(128, 64, true, true);   // A MN-major, B MN-major
-      const uint32_t k_addr = smem_u32(S.k), v_addr = smem_u32(S.v);
-      const uint32_t pt_addr = smem_u32(S.pt), ds_addr = smem_u32(S.dst);
-      bool ok = mbar_wait(&S.kv_full, 0, wait_ns, abort);
-      auto issue_s_dp = [&](int e) -> bool {
-        const int s = e % NS;
-        if (!mbar_wait(&S.full[s], (e / NS) & 1, wait_ns, abort)) return false;
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(S.q[s]), o_addr = smem_u32(S.dout[s]);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + kColS, sdesc(k_addr + kk * 32, 16, 1024), sdesc(q_addr + kk * 32, 16, 1024),
-                 idSS, kk > 0);
-        mma_commit(&S.s_full);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + kColDP, sdesc(v_addr + kk * 32, 16, 1024),
-                 sdesc(o_addr + kk * 32, 16, 1024), idSS, kk > 0);
-        mma_commit(&S.dp_full);
-        return true;
-      };
-      if (ok) ok = issue_s_dp(0);
-      for (int e = 0; ok && e < n; ++e) {
-        const int s = e % NS;
-        if (!mbar_wait(&S.ds_ready, e & 1, wait_ns, abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (e + 1 < n && !issue_s_dp(e + 1)) {
-          ok = false;
-          break;
-        }
-        const uint32_t q_addr = smem_u32(S.q[s]), o_addr = smem_u32(S.dout[s]);
-        // dV += P^T dO ; dK += dS^T Q   (K = 128 queries, 8 steps of 16)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + kColDV, sdesc(pt_addr + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
-                 sdesc(o_addr + kk * 2048, 16384, 1024), idKM, (e > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + kColDK, sdesc(ds_addr + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
-                 sdesc(q_addr + kk * 2048, 16384, 1024), idKM, (e > 0 || kk > 0) ? 1u : 0u);
-        if (e > 0 && !mbar_wait(&S.dq_free, (e - 1) & 1, wait_ns, abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // dQ = dS K   (A = dS^T read MN-major, K = 128 keys)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + kColDQ, sdesc(ds_addr + kk * 2048, kTileBytes, 1024),
-                 sdesc(k_addr + kk * 2048, 16384, 1024), idMM, kk > 0 ? 1u : 0u);
-        mma_commit(&S.dq_full);
-        mma_commit(&S.pds_free);
-        mma_commit(&S.empty[s]);
-      }
-      if (!ok) fail();
-      mma_commit(&S.kv_done);
-      mma_commit(&S.fin);
-      mbar_wait(&S.fin, 0, wait_ns, abort);
     }
   } else {
-    // ---------------- compute warps ----------------
+    regs_increase<kRegsCompute>();
+    // ---------------- compute warpgroups ----------------
+    const int wg = warp >> 2;                    // query-column half of this warpgroup
     const int lg = warp & 3;
-    const int row = lg * 32 + lane;               // key row (S^T, dP^T) / query row (dQ)
+    const int row = lg * 32 + lane;              // key row (S^T, dP^T) / query row (dQ)
     const uint32_t tl = (uint32_t)(lg * 32) << 16;
-    const int j = view_pos(g, it.kview, it.ktile, row);
-    const bool issuer = (warp == 2 && lane == 0);
+    const bool issuer = (warp == 0 && lane == 0);
     bool ok = true;
-    const uint32_t pt_addr = smem_u32(S.pt), ds_addr = smem_u32(S.dst), st_addr = smem_u32(S.stage);
+    const uint32_t pt_addr = smem_u32(S.pt), ds_addr = smem_u32(S.dst);
+    const uint32_t st_addr = smem_u32(S.stage);
+    int gt = 0, n = 0;
+    // query tile whose dQ is still in TMEM (drained after the next tile's dS)
+    int pend_view = 0, pend_tile = 0, pend_bh = 0;
 
-    // dQ of tile e: TMEM -> registers -> fp32 staging -> TMA reduce-add
-    auto drain_dq = [&](int e) -> bool {
-      bool w = mbar_wait(&S.dq_full, e & 1, wait_ns, abort);
+    // dQ of tile t: TMEM -> registers -> fp32 staging -> TMA reduce-add
+    auto drain_dq = [&](int t) -> bool {
+      bool w = mbar_wait(&S.dq_full, t & 1, wait_ns, abort);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
-      uint32_t dq[64];
-      tmem_ld32(tmem + tl + kColDQ, dq);
-      tmem_ld32(tmem + tl + kColDQ + 32, dq + 32);
+      uint32_t dq[32];
+      tmem_ld32(tmem + tl + kColDQ + wg * 32, dq);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&S.dq_free);
-      if (e > 0) {
-        w = mbar_wait(&S.stg_free, (e - 1) & 1, wait_ns, abort);
-        if (!__all_sync(0xffffffffu, w)) return false;
-      }
+      w = mbar_wait(&S.stg_free, (t & 1) ^ 1, wait_ns, abort);
+      if (!__all_sync(0xffffffffu, w)) return false;
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          st_shared_v4(st_addr + h * kTileBytes + swz128(row, ch), dq[h * 32 + ch * 4 + 0],
-                       dq[h * 32 + ch * 4 + 1], dq[h * 32 + ch * 4 + 2], dq[h * 32 + ch * 4 + 3]);
+      for (int ch = 0; ch < 8; ++ch)
+        st_shared_v4(st_addr + wg * kTileBytes + swz128(row, ch), dq[ch * 4 + 0], dq[ch * 4 + 1],
+                     dq[ch * 4 + 2], dq[ch * 4 + 3]);
       fence_async_smem();
       mbar_arrive(&S.stg_full);
       if (issuer) {
-        if (!mbar_wait(&S.stg_full, e & 1, wait_ns, abort)) return false;
-        const QEnt qe = qents[it.qbeg + e];
-        reduce_tile(maps.dq, it.qview, g, qe.qtile, bh, S.stage);
+        if (!mbar_wait(&S.stg_full, t & 1, wait_ns, abort)) return false;
+        reduce_tile(maps.dq, pend_view, g, pend_tile, pend_bh, S.stage);
         bulk_commit();
         bulk_wait_read_all();
         mbar_arrive(&S.stg_free);
@@ -324,118 +383,123 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       return true;
     };
 
-    for (int e = 0; e < n; ++e) {
-      const int s = e % NS;
-      const QEnt qe = qents[it.qbeg + e];
-      bool w = mbar_wait(&S.s_full, e & 1, wait_ns, abort);
-      w = w && mbar_wait(&S.dp_full, e & 1, wait_ns, abort);
-      w = w && mbar_wait(&S.full[s], (e / NS) & 1, wait_ns, abort);
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const Unit x = unit_of(items, u, NH, B, H, nclasses);
+      if (x.bh < 0) continue;
+      const BwdItem& it = x.it;
+      const int cnt = it.qend - it.qbeg;
+      const int j = view_pos(g, it.kview, it.ktile, row);
+      for (int e = 0; e < cnt; ++e, ++gt) {
+        const int s = gt % NS;
+        const QEnt qe = qents[it.qbeg + e];
+        bool w = mbar_wait(&S.s_full, gt & 1, wait_ns, abort);
+        w = w && mbar_wait(&S.dp_full, gt & 1, wait_ns, abort);
+        w = w && mbar_wait(&S.full[s], (gt / NS) & 1, wait_ns, abort);
+        if (gt > 0) w = w && mbar_wait(&S.pds_free, (gt - 1) & 1, wait_ns, abort);
+        if (e == 0 && n > 0) w = w && mbar_wait(&S.kvstg_free, (n - 1) & 1, wait_ns, abort);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool full = (qe.flag == TILE_FULL);
+        int lo = 0, hi = kTile;
+        if (!full) live_rows(g, it.kview, it.qview, it.rule, qe.qtile, j, lo, hi);
+        float sv[64], dp[64];
+        tmem_ld32(tmem + tl + kColS + wg * 64, reinterpret_cast<uint32_t*>(sv));
+        tmem_ld32(tmem + tl + kColS + wg * 64 + 32, reinterpret_cast<uint32_t*>(sv) + 32);
+        tmem_ld32(tmem + tl + kColDP + wg * 64, reinterpret_cast<uint32_t*>(dp));
+        tmem_ld32(tmem + tl + kColDP + wg * 64 + 32, reinterpret_cast<uint32_t*>(dp) + 32);
+        tmem_wait_ld();
+        if (!full) {
+#pragma unroll
+          for (int xk = 0; xk < 64; ++xk)
+            if (wg * 64 + xk < lo || wg * 64 + xk >= hi) sv[xk] = -INFINITY;
+        }
+        const float* l2 = S.l2[s] + wg * 64;
+        const float* dd = S.dd[s] + wg * 64;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const float4 la = *reinterpret_cast<const float4*>(l2 + ch * 8);
+          const float4 lb = *reinterpret_cast<const float4*>(l2 + ch * 8 + 4);
+          const float4 da = *reinterpret_cast<const float4*>(dd + ch * 8);
+          const float4 db = *reinterpret_cast<const float4*>(dd + ch * 8 + 4);
+          const float lv[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+          const float dv8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+          uint32_t pw[4], dw[4];
+#pragma unroll
+          for (int x2 = 0; x2 < 4; ++x2) {
+            const int xk = ch * 8 + x2 * 2;
+            float a0, a1;
+            ffma2(a0, a1, sv[xk], sv[xk + 1], scale_log2, scale_log2, -lv[2 * x2],
+                  -lv[2 * x2 + 1]);
+            const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+            float t0, t1, q0, q1;
+            fadd2(t0, t1, dp[xk], dp[xk + 1], -dv8[2 * x2], -dv8[2 * x2 + 1]);
+            fmul2(q0, q1, p0, p1, t0, t1);
+            pw[x2] = pack_bf16(p0, p1);
+            dw[x2] = pack_bf16(q0, q1);
+          }
+          st_shared_v4(pt_addr + wg * kTileBytes + swz128(row, ch), pw[0], pw[1], pw[2], pw[3]);
+          st_shared_v4(ds_addr + wg * kTileBytes + swz128(row, ch), dw[0], dw[1], dw[2], dw[3]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&S.ds_ready);
+        if (gt > 0 && !drain_dq(gt - 1)) {
+          ok = false;
+          break;
+        }
+        pend_view = it.qview;
+        pend_tile = qe.qtile;
+        pend_bh = x.bh;
+      }
+      if (!ok) break;
+      // ---- end of unit: dK (warpgroup 0) or dV (warpgroup 1) -> reduce-add ----
+      bool w = mbar_wait(&S.kv_done, n & 1, wait_ns, abort);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      int lo = 0, hi = kTile;
-      if (qe.flag != TILE_FULL) live_rows(g, it.kview, it.qview, it.rule, qe.qtile, j, lo, hi);
-      if (e > 0) {
-        w = mbar_wait(&S.pds_free, (e - 1) & 1, wait_ns, abort);
-        if (!__all_sync(0xffffffffu, w)) {
+      uint32_t r[64];
+      tmem_ld32(tmem + tl + (wg ? kColDV : kColDK), r);
+      tmem_ld32(tmem + tl + (wg ? kColDV : kColDK) + 32, r + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&S.acc_free);
+      const uint32_t dst = wg ? ds_addr : pt_addr;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          st_shared_v4(dst + h * kTileBytes + swz128(row, ch), r[h * 32 + ch * 4 + 0],
+                       r[h * 32 + ch * 4 + 1], r[h * 32 + ch * 4 + 2], r[h * 32 + ch * 4 + 3]);
+      fence_async_smem();
+      mbar_arrive(&S.out_full);
+      if (issuer) {
+        if (!mbar_wait(&S.out_full, n & 1, wait_ns, abort)) {
           ok = false;
           break;
         }
+        reduce_tile(maps.dk, it.kview, g, it.ktile, x.bh, S.pt);
+        reduce_tile(maps.dv, it.kview, g, it.ktile, x.bh, S.dst);
+        bulk_commit();
+        bulk_wait_read_all();
+        mbar_arrive(&S.kvstg_free);
       }
-      const float* l2 = S.l2[s];
-      const float* dd = S.dd[s];
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float sv[64], dp[64];
-        tmem_ld32(tmem + tl + kColS + h * 64, reinterpret_cast<uint32_t*>(sv));
-        tmem_ld32(tmem + tl + kColS + h * 64 + 32, reinterpret_cast<uint32_t*>(sv) + 32);
-        tmem_ld32(tmem + tl + kColDP + h * 64, reinterpret_cast<uint32_t*>(dp));
-        tmem_ld32(tmem + tl + kColDP + h * 64 + 32, reinterpret_cast<uint32_t*>(dp) + 32);
-        tmem_wait_ld();
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t pw[4], dw[4];
-#pragma unroll
-          for (int x2 = 0; x2 < 4; ++x2) {
-            float pv[2], dv2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int x = ch * 8 + x2 * 2 + u;   // column within this half
-              const int col = h * 64 + x;          // query column in the tile
-              const bool live = (col >= lo) && (col < hi);
-              const float p = live ? fast_exp2(fmaf(sv[x], scale_log2, -l2[col])) : 0.f;
-              pv[u] = p;
-              dv2[u] = p * (dp[x] - dd[col]);
-            }
-            pw[x2] = pack_bf16(pv[0], pv[1]);
-            dw[x2] = pack_bf16(dv2[0], dv2[1]);
-          }
-          st_shared_v4(pt_addr + h * kTileBytes + swz128(row, ch), pw[0], pw[1], pw[2], pw[3]);
-          st_shared_v4(ds_addr + h * kTileBytes + swz128(row, ch), dw[0], dw[1], dw[2], dw[3]);
-        }
-      }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(&S.ds_ready);
-      if (e > 0 && !drain_dq(e - 1)) {
-        ok = false;
-        break;
-      }
+      ++n;
     }
-    if (ok && n > 0 && !drain_dq(n - 1)) ok = false;
-    if (ok) {
-      // dK, dV of this key tile: TMEM -> fp32 staging (P^T, dS^T buffers) -> reduce-add
-      bool w = mbar_wait(&S.kv_done, 0, wait_ns, abort);
-      if (!__all_sync(0xffffffffu, w)) {
-        ok = false;
-      } else {
-        tc_fence_after();
-        uint32_t r[64];
-        tmem_ld32(tmem + tl + kColDK, r);
-        tmem_ld32(tmem + tl + kColDK + 32, r + 32);
-        tmem_wait_ld();
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
-            st_shared_v4(pt_addr + h * kTileBytes + swz128(row, ch), r[h * 32 + ch * 4 + 0],
-                         r[h * 32 + ch * 4 + 1], r[h * 32 + ch * 4 + 2], r[h * 32 + ch * 4 + 3]);
-        tmem_ld32(tmem + tl + kColDV, r);
-        tmem_ld32(tmem + tl + kColDV + 32, r + 32);
-        tmem_wait_ld();
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
-            st_shared_v4(ds_addr + h * kTileBytes + swz128(row, ch), r[h * 32 + ch * 4 + 0],
-                         r[h * 32 + ch * 4 + 1], r[h * 32 + ch * 4 + 2], r[h * 32 + ch * 4 + 3]);
-        fence_async_smem();
-        mbar_arrive(&S.out_full);
-        if (issuer) {
-          if (mbar_wait(&S.out_full, 0, wait_ns, abort)) {
-            reduce_tile(maps.dk, it.kview, g, it.ktile, bh, S.pt);
-            reduce_tile(maps.dv, it.kview, g, it.ktile, bh, S.dst);
-            bulk_commit();
-          } else {
-            ok = false;
-          }
-        }
-      }
-    }
+    if (ok && gt > 0 && !drain_dq(gt - 1)) ok = false;
     if (!ok) fail();
     if (issuer) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 9) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace
-}  // namespace st
-
-namespace st {
 
 cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, const float* lse,
                    const void* dout, const float* D, float* dq_acc, float* dk_acc,
@@ -456,10 +520,17 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, c
   cudaError_t err =
       cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  dim3 grid(heads_per_class(c), L->dev.n_bwd_items);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int NH = heads_per_class(c);
+  const long long units = (long long)L->dev.n_bwd_items * NH;
+  if (units > 0x7fffffff) return cudaErrorInvalidValue;
+  const int grid = (int)std::min<long long>(units, sms);
   bwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
-      maps, L->geom, (const BwdItem*)L->dev.bwd_items, (const QEnt*)L->dev.q_ents, c.B, c.H,
-      c.nclasses, c.scale * kLog2e, lse, D, c.status, c.wait_ns);
+      maps, L->geom, (const BwdItem*)L->dev.bwd_items, (int)units, NH,
+      (const QEnt*)L->dev.q_ents, c.B, c.H, c.nclasses, c.scale * kLog2e, lse, D, c.status,
+      c.wait_ns);
   return cudaGetLastError();
 }
 

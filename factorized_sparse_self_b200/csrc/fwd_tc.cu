@@ -6,23 +6,28 @@
 // "Per-layer cost": a block-sparse matmul over the pattern's blocks; the
 // milestone page, "The notation", for the attention itself).
 //
-// One CTA = one query tile (128 rows of one head, in its segment's row order)
-// and its key tiles. Warp roles:
-//   warp 0       TMA producer: the Q tile once, then K and V tiles into a
-//                3-stage ring (natural, summary or residue-class view);
-//   warp 1       TMEM owner and MMA issuer: S = Q K^T (M=128, N=128, K=64)
-//                into one of two TMEM S buffers, then O += P V (M=128, N=64,
-//                K=128) into the TMEM O accumulator;
-//   warps 2..5   softmax: thread = query row = TMEM lane. Loads S, applies the
+// Persistent CTAs, two per SM (96 KB shared memory and 256 TMEM columns
+// each, so the two CTAs of an SM interleave their MMA and softmax phases).
+// A CTA walks a strided share of the work units (query tile x head, longest
+// first). Warp roles:
+//   warp 4       TMA producer: each unit's Q tile into one of two Q buffers
+//                (the next unit's Q loads while the current one computes),
+//                K and V tiles into a 2-stage ring (natural, summary or
+//                residue-class view);
+//   warp 5       TMEM owner and MMA issuer: S = Q K^T (M=128, N=128, K=64)
+//                into TMEM, then O += P V with P read from TMEM (A operand)
+//                and V from shared memory (MN-major);
+//   warps 0..3   softmax: thread = query row = TMEM lane. Loads S, applies the
 //                row's live-key interval on PARTIAL tiles, keeps the running
-//                max (rescaling O in TMEM only when the max grows by more
-//                than 2^8) and the running sum, writes P as bf16 into a
-//                128B-swizzled shared tile for the PV MMA; at the end
-//                normalises O, merges with a previous pass if asked, and
-//                stores O (TMA) and LSE.
+//                max (rescaling O in TMEM only when the max grows by more than
+//                2^8) and sum, writes P as bf16 pairs into TMEM; at the end of
+//                a unit normalises O, merges with a previous pass if asked,
+//                and stores O and LSE from registers.
 // Every wait is bounded; a wait that runs out sets the status word, raises
 // the CTA's abort flag, and all roles drain their in-flight work and return.
 #include <math.h>
+
+#include <algorithm>
 
 #include "launch.h"
 #include "tc_common.cuh"
@@ -32,25 +37,25 @@ namespace {
 
 using namespace tc;
 
-constexpr int NS = 3;                     // K/V stages
+constexpr int NS = 2;                       // K/V stages
 constexpr int kTileBytes = kTile * 64 * 2;  // one 128 x 64 bf16 tile
-constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kThreads = 256;  // warpgroup 0: softmax; warpgroup 1: TMA, MMA
+constexpr uint32_t kRegsSoftmax = 200, kRegsIssue = 56;
+static_assert(128 * kRegsSoftmax + 128 * kRegsIssue == kThreads * 128, "register split");
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 struct FwdMaps {
-  CUtensorMap q[3], k[3], v[3], o[3];  // indexed by View
+  CUtensorMap q[3], k[3], v[3];  // indexed by View
 };
 
 struct SmemFwd {
-  uint8_t q[kTileBytes];          // Q tile; later stages the O tile for the store
+  uint8_t q[2][kTileBytes];
   uint8_t k[NS][kTileBytes];
   uint8_t v[NS][kTileBytes];
-  uint8_t p[2][2 * kTileBytes];   // P tiles: keys 0-63 and 64-127 as two K-blocks
-  uint8_t oprev[kTileBytes];      // merge pass: O of the previous pass
-  uint64_t q_full, oprev_full, o_done, stage_done, fin;
-  uint64_t kv_full[NS], kv_empty[NS], s_full[2], p_full[2];
+  uint64_t q_full[2], q_empty[2], kv_full[NS], kv_empty[NS];
+  uint64_t s_full, p_full, pv_done, o_full, o_free, fin;
   uint32_t tmem_base;
   int abort;
 };
@@ -64,16 +69,6 @@ __device__ __forceinline__ void load_tile(void* dst, const CUtensorMap* maps, in
   } else {
     int r = tile / g.ptiles, pb = tile - r * g.ptiles;
     tma_load_4d(dst, &maps[VIEW_CLS], bar, 0, r, pb * kTile, bh);
-  }
-}
-
-__device__ __forceinline__ void store_tile(const CUtensorMap* maps, int view, const Geom& g,
-                                           int tile, int bh, const void* src) {
-  if (view == VIEW_NAT) {
-    tma_store_3d(&maps[VIEW_NAT], src, 0, tile * kTile, bh);
-  } else {
-    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
-    tma_store_4d(&maps[VIEW_CLS], src, 0, r, pb * kTile, bh);
   }
 }
 
@@ -119,278 +114,333 @@ __device__ __forceinline__ void live_cols(const Geom& g, const KeyEnt& ke, int i
   if (hi < lo) hi = lo;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+struct Unit {
+  FwdItem it;
+  int bh;
+};
+
+__device__ __forceinline__ Unit unit_of(const FwdItem* items, int u, int NH, int B, int H,
+                                        int nclasses) {
+  Unit x;
+  x.it = items[u / NH];
+  x.bh = head_of(u % NH, x.it.hclass, B, H, nclasses);
+  return x;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
 fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __restrict__ items,
-              const KeyEnt* __restrict__ keys, int B, int H, int nclasses, float scale_log2,
-              float* __restrict__ lse, int* status, uint64_t wait_ns, int force_timeout) {
+              int n_units, int NH, const KeyEnt* __restrict__ keys, int B, int H, int nclasses,
+              float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+              int* status, uint64_t wait_ns, int force_timeout) {
   extern __shared__ uint8_t smem_raw[];
   SmemFwd& S = *reinterpret_cast<SmemFwd*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
-  const FwdItem it = items[blockIdx.y];
-  const int bh = head_of(blockIdx.x, it.hclass, B, H, nclasses);
-  if (bh < 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n = it.kend - it.kbeg;
   volatile int* abort = &S.abort;
 
   if (threadIdx.x == 0) {
-    mbar_init(&S.q_full, 1);
-    mbar_init(&S.oprev_full, 1);
-    mbar_init(&S.o_done, 1);
-    mbar_init(&S.stage_done, 128);
-    mbar_init(&S.fin, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.q_full[b], 1);
+      mbar_init(&S.q_empty[b], 1);
+    }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&S.kv_full[s], 1);
       mbar_init(&S.kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&S.s_full[b], 1);
-      mbar_init(&S.p_full[b], 128);
-    }
+    mbar_init(&S.s_full, 1);
+    mbar_init(&S.p_full, 128);
+    mbar_init(&S.pv_done, 1);
+    mbar_init(&S.o_full, 1);
+    mbar_init(&S.o_free, 128);
+    mbar_init(&S.fin, 1);
     S.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 5) {
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
-
   auto fail = [&]() {
     *abort = 1;
     set_status(status, ST_ERR_DEVICE_TIMEOUT);
   };
 
-  if (warp == 0) {
+  // Registers: the launch gives 128 per thread; the softmax warpgroup raises
+  // its budget to kRegsSoftmax and the TMA / MMA warpgroup lowers its own to
+  // kRegsIssue (128 * kRegsSoftmax + 128 * kRegsIssue = 256 * 128). Each
+  // role's whole body sits inside the branch that set its budget.
+  if (warp >= 4) {
+    regs_decrease<kRegsIssue>();
+  if (warp == 4) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      int issued[NS];
-      for (int s = 0; s < NS; ++s) issued[s] = -1;
-      mbar_arrive_expect_tx(&S.q_full, kTileBytes);
-      load_tile(S.q, maps.q, it.qview, g, it.qtile, bh, &S.q_full);
-      if (it.merge) {
-        mbar_arrive_expect_tx(&S.oprev_full, kTileBytes);
-        load_tile(S.oprev, maps.o, it.qview, g, it.qtile, bh, &S.oprev_full);
-      }
-      for (int e = 0; e < n; ++e) {
-        const int s = e % NS;
-        if (e >= NS && !mbar_wait(&S.kv_empty[s], ((e / NS) - 1) & 1, wait_ns, abort)) {
-          fail();
+      int kv_last[NS] = {-1, -1};
+      int q_last[2] = {-1, -1};
+      int gt = 0;  // global tile counter of this CTA
+      bool ok = true;
+      int n = 0;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        const Unit x = unit_of(items, u, NH, B, H, nclasses);
+        if (x.bh < 0) continue;
+        const int qb = n & 1;
+        if (!mbar_wait(&S.q_empty[qb], ((n >> 1) & 1) ^ 1, wait_ns, abort)) {
+          ok = false;
           break;
         }
-        if (force_timeout && e == 0) continue;  // test hook: this stage never fills
-        const KeyEnt ke = keys[it.kbeg + e];
-        mbar_arrive_expect_tx(&S.kv_full[s], 2 * kTileBytes);
-        load_tile(S.k[s], maps.k, ke.kview, g, ke.ktile, bh, &S.kv_full[s]);
-        load_tile(S.v[s], maps.v, ke.kview, g, ke.ktile, bh, &S.kv_full[s]);
-        issued[s] = e;
+        mbar_arrive_expect_tx(&S.q_full[qb], kTileBytes);
+        load_tile(S.q[qb], maps.q, x.it.qview, g, x.it.qtile, x.bh, &S.q_full[qb]);
+        q_last[qb] = n;
+        for (int e = x.it.kbeg; e < x.it.kend; ++e, ++gt) {
+          const int s = gt % NS;
+          if (!mbar_wait(&S.kv_empty[s], ((gt / NS) & 1) ^ 1, wait_ns, abort)) {
+            ok = false;
+            break;
+          }
+          if (force_timeout && gt == 0) continue;  // test hook: this stage never fills
+          const KeyEnt ke = keys[e];
+          mbar_arrive_expect_tx(&S.kv_full[s], 2 * kTileBytes);
+          load_tile(S.k[s], maps.k, ke.kview, g, ke.ktile, x.bh, &S.kv_full[s]);
+          load_tile(S.v[s], maps.v, ke.kview, g, ke.ktile, x.bh, &S.kv_full[s]);
+          kv_last[s] = gt;
+        }
+        ++n;
       }
+      if (!ok) fail();
       // no copy may be in flight when the CTA exits
-      mbar_wait(&S.q_full, 0, wait_ns, abort);
-      if (it.merge) mbar_wait(&S.oprev_full, 0, wait_ns, abort);
+      for (int b = 0; b < 2; ++b)
+        if (q_last[b] >= 0 && !mbar_wait(&S.q_full[b], (q_last[b] >> 1) & 1, wait_ns, abort))
+          fail();
       for (int s = 0; s < NS; ++s)
-        if (issued[s] >= 0 && !mbar_wait(&S.kv_full[s], (issued[s] / NS) & 1, wait_ns, abort))
+        if (kv_last[s] >= 0 && !mbar_wait(&S.kv_full[s], (kv_last[s] / NS) & 1, wait_ns, abort))
           fail();
     }
-  } else if (warp == 1) {
+  } else if (warp == 5) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(128, 128, false, false);
       const uint32_t idPV = idesc_bf16(128, 64, false, true);
-      const uint32_t q_addr = smem_u32(S.q);
-      bool ok = mbar_wait(&S.q_full, 0, wait_ns, abort);
-      auto issue_s = [&](int e) -> bool {
-        const int s = e % NS, b = e & 1;
-        if (!mbar_wait(&S.kv_full[s], (e / NS) & 1, wait_ns, abort)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(S.k[s]);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + b * 128, sdesc(q_addr + kk * 32, 16, 1024),
-                 sdesc(k_addr + kk * 32, 16, 1024), idS, kk > 0);
-        mma_commit(&S.s_full[b]);
-        return true;
-      };
-      if (ok && n > 0) ok = issue_s(0);
-      if (ok && n > 1) ok = issue_s(1);
-      for (int e = 0; ok && e < n; ++e) {
-        const int s = e % NS, b = e & 1;
-        if (!mbar_wait(&S.p_full[b], (e >> 1) & 1, wait_ns, abort)) {
+      bool ok = true;
+      int gt = 0, n = 0;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        const Unit x = unit_of(items, u, NH, B, H, nclasses);
+        if (x.bh < 0) continue;
+        const int qb = n & 1;
+        const int cnt = x.it.kend - x.it.kbeg;
+        if (!mbar_wait(&S.q_full[qb], (n >> 1) & 1, wait_ns, abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t p_addr = smem_u32(S.p[b]);
-        const uint32_t v_addr = smem_u32(S.v[s]);
+        const uint32_t q_addr = smem_u32(S.q[qb]);
+        for (int e = 0; e < cnt; ++e, ++gt) {
+          const int s = gt % NS;
+          if (!mbar_wait(&S.kv_full[s], (gt / NS) & 1, wait_ns, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(S.k[s]), v_addr = smem_u32(S.v[s]);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + kColO, sdesc(p_addr + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
-                 sdesc(v_addr + kk * 2048, 16384, 1024), idPV, (e > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&S.o_done);
-        mma_commit(&S.kv_empty[s]);
-        if (e + 2 < n) ok = issue_s(e + 2);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + kColS, sdesc(q_addr + kk * 32, 16, 1024),
+                   sdesc(k_addr + kk * 32, 16, 1024), idS, kk > 0);
+          mma_commit(&S.s_full);
+          if (!mbar_wait(&S.p_full, gt & 1, wait_ns, abort)) {
+            ok = false;
+            break;
+          }
+          if (e == 0 && !mbar_wait(&S.o_free, (n & 1) ^ 1, wait_ns, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + kColO, tmem + kColP + kk * 8, sdesc(v_addr + kk * 2048, 16384, 1024),
+                   idPV, (e > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&S.pv_done);
+          mma_commit(&S.kv_empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&S.q_empty[qb]);
+        mma_commit(&S.o_full);
+        ++n;
       }
       if (!ok) fail();
       mma_commit(&S.fin);
       mbar_wait(&S.fin, 0, wait_ns, abort);
     }
+  }
   } else {
+    regs_increase<kRegsSoftmax>();
     // ---------------- softmax warps ----------------
-    const int lg = warp & 3;                 // TMEM lane group of this warp
-    const int row = lg * 32 + lane;          // query row in the tile = TMEM lane
+    const int lg = warp;              // TMEM lane group of this warp
+    const int row = lg * 32 + lane;   // query row in the tile = TMEM lane
     const uint32_t tl = (uint32_t)(lg * 32) << 16;
-    const int i = view_pos(g, it.qview, it.qtile, row);
-    float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int e = 0; e < n; ++e) {
-      const int b = e & 1;
-      const KeyEnt ke = keys[it.kbeg + e];
-      ok = mbar_wait(&S.s_full[b], (e >> 1) & 1, wait_ns, abort);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      float s[128];
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4)
-        tmem_ld32(tmem + tl + b * 128 + c4 * 32, reinterpret_cast<uint32_t*>(s) + c4 * 32);
-      tmem_wait_ld();
-      if (ke.flag != TILE_FULL) {
-        int lo, hi;
-        live_cols(g, ke, i, lo, hi);
-#pragma unroll
-        for (int x = 0; x < 128; ++x)
-          if (x < lo || x >= hi) s[x] = -INFINITY;
-      }
-      float mt = s[0];
-#pragma unroll
-      for (int x = 1; x < 128; ++x) mt = fmaxf(mt, s[x]);
-      mt *= scale_log2;
-      const float m_new = fmaxf(m_run, mt);
-      float alpha = 1.f;
-      bool rescale_o = false;
-      if (m_new > m_run + kRescaleThreshold) {
-        rescale_o = (m_run != -INFINITY);
-        alpha = fast_exp2(m_run - m_new);
-        m_run = m_new;
-      }
-      const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-      float rs = 0.f;
-      const uint32_t pb = smem_u32(S.p[b]);
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        float p8[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          p8[x] = fast_exp2(fmaf(s[ch * 8 + x], scale_log2, -mu));
-          rs += p8[x];
-        }
-        st_shared_v4(pb + (ch >> 3) * kTileBytes + swz128(row, ch & 7), pack_bf16(p8[0], p8[1]),
-                     pack_bf16(p8[2], p8[3]), pack_bf16(p8[4], p8[5]), pack_bf16(p8[6], p8[7]));
-      }
-      l_run = l_run * alpha + rs;
-      if (e > 0) {
-        ok = mbar_wait(&S.o_done, (e - 1) & 1, wait_ns, abort);
-        ok = __all_sync(0xffffffffu, ok);
+    int gt = 0, n = 0;
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const Unit x = unit_of(items, u, NH, B, H, nclasses);
+      if (x.bh < 0) continue;
+      const FwdItem& it = x.it;
+      const int bh = x.bh;
+      const int i = view_pos(g, it.qview, it.qtile, row);
+      const int cnt = it.kend - it.kbeg;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int e = 0; e < cnt; ++e, ++gt) {
+        const KeyEnt ke = keys[it.kbeg + e];
+        ok = __all_sync(0xffffffffu, mbar_wait(&S.s_full, gt & 1, wait_ns, abort));
         if (!ok) break;
         tc_fence_after();
+        // S is read from TMEM twice, 64 columns at a time (max, then exp), to
+        // keep the live registers within the two-CTAs-per-SM budget. FULL
+        // tiles skip the per-element mask.
+        const bool full = (ke.flag == TILE_FULL);
+        int lo = 0, hi = kTile;
+        if (!full) live_cols(g, ke, i, lo, hi);
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          float s[64];
+          tmem_ld32(tmem + tl + kColS + h * 64, reinterpret_cast<uint32_t*>(s));
+          tmem_ld32(tmem + tl + kColS + h * 64 + 32, reinterpret_cast<uint32_t*>(s) + 32);
+          tmem_wait_ld();
+          if (!full) {
+#pragma unroll
+            for (int xk = 0; xk < 64; ++xk)
+              if (h * 64 + xk < lo || h * 64 + xk >= hi) s[xk] = -INFINITY;
+          }
+#pragma unroll
+          for (int xk = 0; xk < 64; xk += 8) {
+            m4[0] = fmax3(m4[0], s[xk + 0], s[xk + 1]);
+            m4[1] = fmax3(m4[1], s[xk + 2], s[xk + 3]);
+            m4[2] = fmax3(m4[2], s[xk + 4], s[xk + 5]);
+            m4[3] = fmax3(m4[3], s[xk + 6], s[xk + 7]);
+          }
+        }
+        const float mt = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * scale_log2;
+        const float m_new = fmaxf(m_run, mt);
+        float alpha = 1.f;
+        bool rescale_o = false;
+        if (m_new > m_run + kRescaleThreshold) {
+          rescale_o = (m_run != -INFINITY);
+          alpha = fast_exp2(m_run - m_new);
+          m_run = m_new;
+        }
+        const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+        if (gt > 0) {
+          // PV of the previous tile is done: P may be overwritten, O is stable
+          ok = __all_sync(0xffffffffu, mbar_wait(&S.pv_done, (gt - 1) & 1, wait_ns, abort));
+          if (!ok) break;
+          tc_fence_after();
+        }
         if (__any_sync(0xffffffffu, rescale_o)) {
           const float a = rescale_o ? alpha : 1.f;
-#pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            uint32_t o[32];
-            tmem_ld32(tmem + tl + kColO + c2 * 32, o);
+#pragma unroll 1
+          for (int c8 = 0; c8 < 8; ++c8) {
+            uint32_t o[8];
+            tmem_ld8(tmem + tl + kColO + c8 * 8, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * a);
-            tmem_st32(tmem + tl + kColO + c2 * 32, o);
+            for (int xk = 0; xk < 8; ++xk) o[xk] = __float_as_uint(__uint_as_float(o[xk]) * a);
+            tmem_st8(tmem + tl + kColO + c8 * 8, o);
           }
-          tmem_wait_st();
         }
-      }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(&S.p_full[b]);
-    }
-    if (!ok) {
-      fail();
-    } else {
-      // ---- epilogue ----
-      float out[64];
-      if (n > 0) {
-        ok = mbar_wait(&S.o_done, (n - 1) & 1, wait_ns, abort);
-        ok = __all_sync(0xffffffffu, ok);
-      }
-      if (ok && it.merge) ok = __all_sync(0xffffffffu, mbar_wait(&S.oprev_full, 0, wait_ns, abort));
-      if (!ok) {
-        fail();
-      } else {
-        if (n > 0) {
-          tc_fence_after();
-          tmem_ld32(tmem + tl + kColO, reinterpret_cast<uint32_t*>(out));
-          tmem_ld32(tmem + tl + kColO + 32, reinterpret_cast<uint32_t*>(out) + 32);
+        // exp pass: one packed FMA forms two exponents, masked entries are -inf
+        // and give exactly 0; four pairs of partial sums break the add chain.
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        const float nmu = -mu;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          float s[64];
+          tmem_ld32(tmem + tl + kColS + h * 64, reinterpret_cast<uint32_t*>(s));
+          tmem_ld32(tmem + tl + kColS + h * 64 + 32, reinterpret_cast<uint32_t*>(s) + 32);
           tmem_wait_ld();
-        }
-        const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-        float L = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+          if (!full) {
 #pragma unroll
-        for (int x = 0; x < 64; ++x) out[x] = (n > 0) ? out[x] * inv : 0.f;
-        if (it.merge && i >= 0) {
-          const float Lp = lse[(size_t)bh * g.T + i];
-          const float mx = fmaxf(Lp, L);
-          float wp = 0.f, wc = 0.f;
-          if (mx != -INFINITY) {
-            const float Ln = mx + __logf(__expf(Lp - mx) + __expf(L - mx));
-            wp = __expf(Lp - Ln);
-            wc = __expf(L - Ln);
-            L = Ln;
+            for (int xk = 0; xk < 64; ++xk)
+              if (h * 64 + xk < lo || h * 64 + xk >= hi) s[xk] = -INFINITY;
           }
-          const uint32_t ob = smem_u32(S.oprev);
+          uint32_t pk[32];
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            uint32_t w[4];
-            ld_shared_v4(ob + swz128(row, ch), w[0], w[1], w[2], w[3]);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&w[x]);
-              float2 f = __bfloat1622float2(h);
-              out[ch * 8 + 2 * x] = fmaf(wp, f.x, wc * out[ch * 8 + 2 * x]);
-              out[ch * 8 + 2 * x + 1] = fmaf(wp, f.y, wc * out[ch * 8 + 2 * x + 1]);
-            }
+          for (int xk = 0; xk < 64; xk += 2) {
+            float a0, a1;
+            ffma2(a0, a1, s[xk], s[xk + 1], scale_log2, scale_log2, nmu, nmu);
+            const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+            const int j = (xk >> 1) & 3;
+            fadd2(sa[j], sb[j], sa[j], sb[j], p0, p1);
+            pk[xk >> 1] = pack_bf16(p0, p1);
           }
+          tmem_st32(tmem + tl + kColP + h * 32, pk);
         }
-        const uint32_t qb = smem_u32(S.q);  // Q is no longer read: stage O here
+        l_run = l_run * alpha + (((sa[0] + sb[0]) + (sa[1] + sb[1])) +
+                                 ((sa[2] + sb[2]) + (sa[3] + sb[3])));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&S.p_full);
+      }
+      if (!ok) break;
+      // ---- epilogue of the unit ----
+      ok = __all_sync(0xffffffffu, mbar_wait(&S.o_full, n & 1, wait_ns, abort));
+      if (!ok) break;
+      tc_fence_after();
+      float o[64];
+      if (cnt > 0) {
+        tmem_ld32(tmem + tl + kColO, reinterpret_cast<uint32_t*>(o));
+        tmem_ld32(tmem + tl + kColO + 32, reinterpret_cast<uint32_t*>(o) + 32);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(&S.o_free);
+      ++n;
+      if (i < 0) continue;
+      const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      float L = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          st_shared_v4(qb + swz128(row, ch), pack_bf16(out[ch * 8 + 0], out[ch * 8 + 1]),
-                       pack_bf16(out[ch * 8 + 2], out[ch * 8 + 3]),
-                       pack_bf16(out[ch * 8 + 4], out[ch * 8 + 5]),
-                       pack_bf16(out[ch * 8 + 6], out[ch * 8 + 7]));
-        if (i >= 0) lse[(size_t)bh * g.T + i] = L;
-        fence_async_smem();
-        mbar_arrive(&S.stage_done);
-        if (warp == 2 && lane == 0) {
-          if (mbar_wait(&S.stage_done, 0, wait_ns, abort)) {
-            store_tile(maps.o, it.qview, g, it.qtile, bh, S.q);
-            bulk_commit();
-            bulk_wait_all();
-          } else {
-            fail();
+      for (int xk = 0; xk < 64; ++xk) o[xk] = (cnt > 0) ? o[xk] * inv : 0.f;
+      const size_t rowoff = ((size_t)bh * g.T + i) * 64;
+      uint4* dst = reinterpret_cast<uint4*>(out + rowoff);
+      if (it.merge) {
+        const float Lp = lse[(size_t)bh * g.T + i];
+        const float mx2 = fmaxf(Lp, L);
+        float wp = 0.f, wc = 0.f;
+        if (mx2 != -INFINITY) {
+          const float Ln = mx2 + __logf(__expf(Lp - mx2) + __expf(L - mx2));
+          wp = __expf(Lp - Ln);
+          wc = __expf(L - Ln);
+          L = Ln;
+        }
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint4 w = dst[ch];
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ws[q2]));
+            o[ch * 8 + 2 * q2] = fmaf(wp, f.x, wc * o[ch * 8 + 2 * q2]);
+            o[ch * 8 + 2 * q2 + 1] = fmaf(wp, f.y, wc * o[ch * 8 + 2 * q2 + 1]);
           }
         }
       }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        dst[ch] = make_uint4(pack_bf16(o[ch * 8 + 0], o[ch * 8 + 1]),
+                             pack_bf16(o[ch * 8 + 2], o[ch * 8 + 3]),
+                             pack_bf16(o[ch * 8 + 4], o[ch * 8 + 5]),
+                             pack_bf16(o[ch * 8 + 6], o[ch * 8 + 7]));
+      lse[(size_t)bh * g.T + i] = L;
     }
+    if (!ok) fail();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace
-}  // namespace st
-
-namespace st {
 
 cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, void* o,
                    float* lse, int force_timeout) {
@@ -399,22 +449,27 @@ cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, v
   FwdMaps maps;
   if (!make_view_maps(maps.q, q, false, L->geom, BH, c.d) ||
       !make_view_maps(maps.k, k, false, L->geom, BH, c.d) ||
-      !make_view_maps(maps.v, v, false, L->geom, BH, c.d) ||
-      !make_view_maps(maps.o, o, false, L->geom, BH, c.d))
+      !make_view_maps(maps.v, v, false, L->geom, BH, c.d))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(SmemFwd) + 1024;
   cudaError_t err =
       cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const float scale_log2 = c.scale * 1.4426950408889634f;
+  const int NH = heads_per_class(c);
   for (int pass = 0; pass < L->n_passes; ++pass) {
     const int n = L->dev.n_fwd_items[pass];
     if (n == 0) continue;
-    dim3 grid(heads_per_class(c), n);
+    const long long units = (long long)n * NH;
+    if (units > 0x7fffffff) return cudaErrorInvalidValue;
+    const int grid = (int)std::min<long long>(units, 2LL * sms);
     fwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
-        maps, L->geom, (const FwdItem*)L->dev.fwd_items[pass], (const KeyEnt*)L->dev.key_ents,
-        c.B, c.H, c.nclasses, scale_log2, lse, c.status, c.wait_ns,
-        (force_timeout && pass == 0) ? 1 : 0);
+        maps, L->geom, (const FwdItem*)L->dev.fwd_items[pass], (int)units, NH,
+        (const KeyEnt*)L->dev.key_ents, c.B, c.H, c.nclasses, scale_log2, (__nv_bfloat16*)o, lse,
+        c.status, c.wait_ns, (force_timeout && pass == 0) ? 1 : 0);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }

@@ -326,7 +326,18 @@ st_status build_layout(const st_pattern_desc* desc, st_layout* L) {
         p.it.kview = s.kview;
         p.it.qview = s.qview;
         p.it.rule = s.rule;
-        bitems.push_back(std::move(p));
+        // Long key columns (summary keys are read by every later query tile)
+        // are cut into chunks so that no CTA carries a whole column; each
+        // chunk reduce-adds its own dK, dV partial.
+        const size_t nq = p.qs.size();
+        const size_t nchunks = (nq + kBwdChunk - 1) / kBwdChunk;
+        for (size_t ch = 0; ch < nchunks; ++ch) {
+          const size_t a = nq * ch / nchunks, b = nq * (ch + 1) / nchunks;
+          PendingB part;
+          part.it = p.it;
+          part.qs.assign(p.qs.begin() + a, p.qs.begin() + b);
+          bitems.push_back(std::move(part));
+        }
       }
     }
   }

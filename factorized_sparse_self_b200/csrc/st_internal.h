@@ -10,6 +10,7 @@
 namespace st {
 
 constexpr int kTile = 128;  // query and key tile edge, in view rows
+constexpr int kBwdChunk = 8; // most query tiles one backward work item visits
 
 // Row orders ("views") a segment reads its queries or keys in.
 enum View : uint8_t {
