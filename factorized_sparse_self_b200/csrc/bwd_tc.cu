@@ -517,21 +517,29 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, c
       !make_view_maps(maps.dv, dv_acc, true, L->geom, BH, c.d))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(SmemBwd) + 1024;
-  cudaError_t err =
-      cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
-  int dev = 0, sms = 148;
+  static bool attr_set[64] = {false};
+  int dev = 0;
   cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaError_t err = cudaSuccess;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    err = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+    if (err != cudaSuccess) return err;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  const int sms = sm_count();
   const int NH = heads_per_class(c);
   const long long units = (long long)L->dev.n_bwd_items * NH;
   if (units > 0x7fffffff) return cudaErrorInvalidValue;
   const int grid = (int)std::min<long long>(units, sms);
+  record_begin(c);
   bwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
       maps, L->geom, (const BwdItem*)L->dev.bwd_items, (int)units, NH,
       (const QEnt*)L->dev.q_ents, c.B, c.H, c.nclasses, c.scale * kLog2e, lse, D, c.status,
       c.wait_ns);
-  return cudaGetLastError();
+  err = cudaGetLastError();
+  record_end(c);
+  return err;
 }
 
 }  // namespace st

@@ -110,10 +110,12 @@ bool g_timing = false;
 cudaEvent_t g_ev[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
 bool g_ev_used[2] = {false, false};
 
-void mark(int kernel, int which, cudaStream_t s) {
+// Hands the benchmark events of `kernel` to a call (when timing is on).
+void arm(Call& c, int kernel) {
   if (!g_timing) return;
-  cudaEventRecord(g_ev[kernel][which], s);
-  if (which == 1) g_ev_used[kernel] = true;
+  c.ev_begin = g_ev[kernel][0];
+  c.ev_end = g_ev[kernel][1];
+  g_ev_used[kernel] = true;
 }
 
 }  // namespace
@@ -262,7 +264,7 @@ st_status st_sparse_attn_fwd(const st_layout* L, st_dtype dtype, int32_t B, int3
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return ST_ERR_INVALID;
   cudaError_t e;
-  mark(0, 0, c.stream);
+  arm(c, 0);
   if (dtype == ST_F32) {
     e = simt_fwd(c, q, k, v, o, lse);
   } else {
@@ -270,7 +272,6 @@ st_status st_sparse_attn_fwd(const st_layout* L, st_dtype dtype, int32_t B, int3
     g_force_timeout = 0;
     e = tc_fwd(c, q, k, v, o, lse, ft);
   }
-  mark(0, 1, c.stream);
   return e == cudaSuccess ? ST_OK : ST_ERR_CUDA;
 }
 
@@ -308,10 +309,10 @@ st_status st_sparse_attn_bwd(const st_layout* L, st_dtype dtype, int32_t B, int3
     if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, elems * sizeof(float), c.stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, elems * sizeof(float), c.stream);
     if (e == cudaSuccess) e = bwd_prologue(c, o, dout, Dv, nullptr, 0);
-    mark(1, 0, c.stream);
+    Call cm = c;
+    arm(cm, 1);
     if (e == cudaSuccess)
-      e = simt_bwd(c, q, k, v, lse, dout, Dv, (float*)dq, (float*)dk, (float*)dv);
-    mark(1, 1, c.stream);
+      e = simt_bwd(cm, q, k, v, lse, dout, Dv, (float*)dq, (float*)dk, (float*)dv);
   } else {
     float* acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
                                           round256(rows * sizeof(float)));
@@ -319,10 +320,10 @@ st_status st_sparse_attn_bwd(const st_layout* L, st_dtype dtype, int32_t B, int3
     // the three accumulators must be back to back for the epilogue
     if (stride != elems) return ST_ERR_UNSUPPORTED;
     e = bwd_prologue(c, o, dout, Dv, acc, 3 * elems);
-    mark(1, 0, c.stream);
+    Call cm = c;
+    arm(cm, 1);
     if (e == cudaSuccess)
-      e = tc_bwd(c, q, k, v, lse, dout, Dv, acc, acc + stride, acc + 2 * stride);
-    mark(1, 1, c.stream);
+      e = tc_bwd(cm, q, k, v, lse, dout, Dv, acc, acc + stride, acc + 2 * stride);
     if (e == cudaSuccess) e = bwd_epilogue(c, acc, dq, dk, dv, elems);
   }
   return e == cudaSuccess ? ST_OK : ST_ERR_CUDA;

@@ -40,7 +40,7 @@ using namespace tc;
 constexpr int NS = 2;                       // K/V stages
 constexpr int kTileBytes = kTile * 64 * 2;  // one 128 x 64 bf16 tile
 constexpr int kThreads = 256;  // warpgroup 0: softmax; warpgroup 1: TMA, MMA
-constexpr uint32_t kRegsSoftmax = 200, kRegsIssue = 56;
+constexpr uint32_t kRegsSoftmax = 216, kRegsIssue = 40;
 static_assert(128 * kRegsSoftmax + 128 * kRegsIssue == kThreads * 128, "register split");
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
@@ -55,7 +55,7 @@ struct SmemFwd {
   uint8_t k[NS][kTileBytes];
   uint8_t v[NS][kTileBytes];
   uint64_t q_full[2], q_empty[2], kv_full[NS], kv_empty[NS];
-  uint64_t s_full, p_full, pv_done, o_full, o_free, fin;
+  uint64_t s_full, s_free, p_full, pv_done, o_full, o_free, fin;
   uint32_t tmem_base;
   int abort;
 };
@@ -148,6 +148,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       mbar_init(&S.kv_empty[s], 1);
     }
     mbar_init(&S.s_full, 1);
+    mbar_init(&S.s_free, 128);
     mbar_init(&S.p_full, 128);
     mbar_init(&S.pv_done, 1);
     mbar_init(&S.o_full, 1);
@@ -223,31 +224,76 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       const uint32_t idS = idesc_bf16(128, 128, false, false);
       const uint32_t idPV = idesc_bf16(128, 64, false, true);
       bool ok = true;
-      int gt = 0, n = 0;
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-        const Unit x = unit_of(items, u, NH, B, H, nclasses);
-        if (x.bh < 0) continue;
+      int gt = 0, n = 0;  // tiles and units of this CTA issued so far
+      // S of global tile g from Q buffer qb and K ring stage g % NS.
+      auto issue_s = [&](int g, int qb) -> bool {
+        const int s = g % NS;
+        if (!mbar_wait(&S.kv_full[s], (g / NS) & 1, wait_ns, abort)) return false;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(S.q[qb]), k_addr = smem_u32(S.k[s]);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem + kColS, sdesc(q_addr + kk * 32, 16, 1024),
+                 sdesc(k_addr + kk * 32, 16, 1024), idS, kk > 0);
+        mma_commit(&S.s_full);
+        return true;
+      };
+      // first unit at or after u with a valid head
+      auto seek = [&](int u, Unit& x) -> int {
+        for (; u < n_units; u += gridDim.x) {
+          x = unit_of(items, u, NH, B, H, nclasses);
+          if (x.bh >= 0) return u;
+        }
+        return n_units;
+      };
+      Unit cur;
+      int u = seek(blockIdx.x, cur);
+      bool first_done = false;  // S of this unit's first tile already issued ahead
+      while (ok && u < n_units) {
         const int qb = n & 1;
-        const int cnt = x.it.kend - x.it.kbeg;
+        const int cnt = cur.it.kend - cur.it.kbeg;
         if (!mbar_wait(&S.q_full[qb], (n >> 1) & 1, wait_ns, abort)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(S.q[qb]);
-        for (int e = 0; e < cnt; ++e, ++gt) {
-          const int s = gt % NS;
-          if (!mbar_wait(&S.kv_full[s], (gt / NS) & 1, wait_ns, abort)) {
+        if (cnt > 0 && !first_done) {
+          if (gt > 0 && !mbar_wait(&S.s_free, (gt - 1) & 1, wait_ns, abort)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(S.k[s]), v_addr = smem_u32(S.v[s]);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + kColS, sdesc(q_addr + kk * 32, 16, 1024),
-                   sdesc(k_addr + kk * 32, 16, 1024), idS, kk > 0);
-          mma_commit(&S.s_full);
+          if (!issue_s(gt, qb)) {
+            ok = false;
+            break;
+          }
+        }
+        first_done = false;
+        Unit nx;
+        const int un = seek(u + gridDim.x, nx);
+        for (int e = 0; e < cnt; ++e, ++gt) {
+          const int s = gt % NS;
+          // S of the next tile (this unit's, or the first of the next unit) goes
+          // out as soon as the softmax has read S of this one, ahead of PV.
+          const bool next_here = (e + 1 < cnt);
+          const bool next_unit = !next_here && un < n_units && nx.it.kend > nx.it.kbeg;
+          if (next_here || next_unit) {
+            if (!mbar_wait(&S.s_free, gt & 1, wait_ns, abort)) {
+              ok = false;
+              break;
+            }
+            int nqb = qb;
+            if (next_unit) {
+              nqb = (n + 1) & 1;
+              if (!mbar_wait(&S.q_full[nqb], ((n + 1) >> 1) & 1, wait_ns, abort)) {
+                ok = false;
+                break;
+              }
+            }
+            if (!issue_s(gt + 1, nqb)) {
+              ok = false;
+              break;
+            }
+            if (next_unit) first_done = true;
+          }
           if (!mbar_wait(&S.p_full, gt & 1, wait_ns, abort)) {
             ok = false;
             break;
@@ -257,6 +303,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
             break;
           }
           tc_fence_after();
+          const uint32_t v_addr = smem_u32(S.v[s]);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + kColO, tmem + kColP + kk * 8, sdesc(v_addr + kk * 2048, 16384, 1024),
@@ -268,6 +315,8 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         mma_commit(&S.q_empty[qb]);
         mma_commit(&S.o_full);
         ++n;
+        u = un;
+        cur = nx;
       }
       if (!ok) fail();
       mma_commit(&S.fin);
@@ -295,31 +344,31 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         ok = __all_sync(0xffffffffu, mbar_wait(&S.s_full, gt & 1, wait_ns, abort));
         if (!ok) break;
         tc_fence_after();
-        // S is read from TMEM twice, 64 columns at a time (max, then exp), to
-        // keep the live registers within the two-CTAs-per-SM budget. FULL
-        // tiles skip the per-element mask.
+        // S is read from TMEM once; the buffer is released at once so the MMA
+        // warp can compute the next tile's S while this one is exponentiated.
+        // FULL tiles skip the per-element mask.
+        float s[128];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+          tmem_ld32(tmem + tl + kColS + c4 * 32, reinterpret_cast<uint32_t*>(s) + c4 * 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&S.s_free);
         const bool full = (ke.flag == TILE_FULL);
-        int lo = 0, hi = kTile;
-        if (!full) live_cols(g, ke, i, lo, hi);
+        if (!full) {
+          int lo, hi;
+          live_cols(g, ke, i, lo, hi);
+#pragma unroll
+          for (int xk = 0; xk < 128; ++xk)
+            if (xk < lo || xk >= hi) s[xk] = -INFINITY;
+        }
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          float s[64];
-          tmem_ld32(tmem + tl + kColS + h * 64, reinterpret_cast<uint32_t*>(s));
-          tmem_ld32(tmem + tl + kColS + h * 64 + 32, reinterpret_cast<uint32_t*>(s) + 32);
-          tmem_wait_ld();
-          if (!full) {
 #pragma unroll
-            for (int xk = 0; xk < 64; ++xk)
-              if (h * 64 + xk < lo || h * 64 + xk >= hi) s[xk] = -INFINITY;
-          }
-#pragma unroll
-          for (int xk = 0; xk < 64; xk += 8) {
-            m4[0] = fmax3(m4[0], s[xk + 0], s[xk + 1]);
-            m4[1] = fmax3(m4[1], s[xk + 2], s[xk + 3]);
-            m4[2] = fmax3(m4[2], s[xk + 4], s[xk + 5]);
-            m4[3] = fmax3(m4[3], s[xk + 6], s[xk + 7]);
-          }
+        for (int xk = 0; xk < 128; xk += 8) {
+          m4[0] = fmax3(m4[0], s[xk + 0], s[xk + 1]);
+          m4[1] = fmax3(m4[1], s[xk + 2], s[xk + 3]);
+          m4[2] = fmax3(m4[2], s[xk + 4], s[xk + 5]);
+          m4[3] = fmax3(m4[3], s[xk + 6], s[xk + 7]);
         }
         const float mt = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * scale_log2;
         const float m_new = fmaxf(m_run, mt);
@@ -353,28 +402,19 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         // and give exactly 0; four pairs of partial sums break the add chain.
         float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
         const float nmu = -mu;
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          float s[64];
-          tmem_ld32(tmem + tl + kColS + h * 64, reinterpret_cast<uint32_t*>(s));
-          tmem_ld32(tmem + tl + kColS + h * 64 + 32, reinterpret_cast<uint32_t*>(s) + 32);
-          tmem_wait_ld();
-          if (!full) {
 #pragma unroll
-            for (int xk = 0; xk < 64; ++xk)
-              if (h * 64 + xk < lo || h * 64 + xk >= hi) s[xk] = -INFINITY;
-          }
-          uint32_t pk[32];
+        for (int h = 0; h < 8; ++h) {
+          uint32_t pk[8];  // 16 keys at a time keeps the live set near S itself
 #pragma unroll
-          for (int xk = 0; xk < 64; xk += 2) {
+          for (int xk = 0; xk < 16; xk += 2) {
             float a0, a1;
-            ffma2(a0, a1, s[xk], s[xk + 1], scale_log2, scale_log2, nmu, nmu);
+            ffma2(a0, a1, s[h * 16 + xk], s[h * 16 + xk + 1], scale_log2, scale_log2, nmu, nmu);
             const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
             const int j = (xk >> 1) & 3;
             fadd2(sa[j], sb[j], sa[j], sb[j], p0, p1);
             pk[xk >> 1] = pack_bf16(p0, p1);
           }
-          tmem_st32(tmem + tl + kColP + h * 32, pk);
+          tmem_st8(tmem + tl + kColP + h * 8, pk);
         }
         l_run = l_run * alpha + (((sa[0] + sb[0]) + (sa[1] + sb[1])) +
                                  ((sa[2] + sb[2]) + (sa[3] + sb[3])));
@@ -452,14 +492,20 @@ cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, v
       !make_view_maps(maps.v, v, false, L->geom, BH, c.d))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(SmemFwd) + 1024;
-  cudaError_t err =
-      cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
-  int dev = 0, sms = 148;
+  static bool attr_set[64] = {false};
+  int dev = 0;
   cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaError_t err = cudaSuccess;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    err = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+    if (err != cudaSuccess) return err;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  const int sms = sm_count();
   const float scale_log2 = c.scale * 1.4426950408889634f;
   const int NH = heads_per_class(c);
+  record_begin(c);
   for (int pass = 0; pass < L->n_passes; ++pass) {
     const int n = L->dev.n_fwd_items[pass];
     if (n == 0) continue;
@@ -473,6 +519,7 @@ cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, v
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
+  record_end(c);
   return cudaSuccess;
 }
 

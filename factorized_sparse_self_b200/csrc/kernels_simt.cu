@@ -306,6 +306,7 @@ cudaError_t simt_fwd_t(const Call& c, const void* q, const void* k, const void* 
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;
+  record_begin(c);
   for (int pass = 0; pass < L->n_passes; ++pass) {
     int n = L->dev.n_fwd_items[pass];
     if (n == 0) continue;
@@ -316,6 +317,7 @@ cudaError_t simt_fwd_t(const Call& c, const void* q, const void* k, const void* 
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
+  record_end(c);
   return cudaSuccess;
 }
 
@@ -333,6 +335,7 @@ cudaError_t simt_bwd_t(const Call& c, const void* q, const void* k, const void* 
   if (err != cudaSuccess) return err;
   err = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_q);
   if (err != cudaSuccess) return err;
+  record_begin(c);
   if (L->dev.n_bwd_items > 0) {
     dim3 grid(heads_per_class(c), L->dev.n_bwd_items);
     kv<<<grid, kThreads, smem_kv, c.stream>>>(
@@ -353,6 +356,7 @@ cudaError_t simt_bwd_t(const Call& c, const void* q, const void* k, const void* 
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
+  record_end(c);
   return cudaSuccess;
 }
 

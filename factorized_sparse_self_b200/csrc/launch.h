@@ -16,7 +16,20 @@ struct Call {
   int* status;      // device status word
   uint64_t wait_ns; // bound of every on-device wait
   cudaStream_t stream;
+  // Benchmark events recorded right before the first and right after the
+  // last attention launch of the call (null when timing is off).
+  cudaEvent_t ev_begin = nullptr, ev_end = nullptr;
 };
+
+inline void record_begin(const Call& c) {
+  if (c.ev_begin) cudaEventRecord(c.ev_begin, c.stream);
+}
+inline void record_end(const Call& c) {
+  if (c.ev_end) cudaEventRecord(c.ev_end, c.stream);
+}
+
+// Multiprocessor count of the current device (queried once per device).
+int sm_count();
 
 // Exact fp32 path (CUDA cores): float32 tensors, d = 32 or 64.
 cudaError_t simt_fwd(const Call& c, const void* q, const void* k, const void* v, void* o,

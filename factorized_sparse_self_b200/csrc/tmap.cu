@@ -1,7 +1,12 @@
 // TMA tensor-map encoding for the three row orders of a [B*H, T, d] tensor.
 // cuTensorMapEncodeTiled is reached through cudaGetDriverEntryPoint, so the
-// library needs no link against the driver library.
+// library needs no link against the driver library. Encoded maps are cached
+// per (address, shape): calls that reuse their buffers (training loops,
+// benchmarks) skip the encoding.
 #include <cuda.h>
+
+#include <cstring>
+#include <mutex>
 
 #include "launch.h"
 
@@ -26,10 +31,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-}  // namespace
-
-bool make_view_maps(CUtensorMap out[3], const void* base, bool is_f32, const Geom& g, int BH,
-                    int d) {
+bool encode_views(CUtensorMap out[3], const void* base, bool is_f32, const Geom& g, int BH,
+                  int d) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const CUtensorMapDataType dt =
@@ -67,6 +70,74 @@ bool make_view_maps(CUtensorMap out[3], const void* base, bool is_f32, const Geo
     }
   }
   return true;
+}
+
+struct Key {
+  const void* base;
+  int is_f32, T, l, c, P, nsum, BH, d;
+  bool operator==(const Key& o) const { return std::memcmp(this, &o, sizeof(Key)) == 0; }
+};
+
+struct Entry {
+  Key key;
+  CUtensorMap maps[3];
+  uint64_t stamp;
+  bool valid;
+};
+
+constexpr int kCacheSize = 64;
+Entry g_cache[kCacheSize];
+uint64_t g_clock = 0;
+std::mutex g_cache_mu;
+
+}  // namespace
+
+bool make_view_maps(CUtensorMap out[3], const void* base, bool is_f32, const Geom& g, int BH,
+                    int d) {
+  Key key;
+  std::memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.is_f32 = is_f32 ? 1 : 0;
+  key.T = g.T;
+  key.l = g.l;
+  key.c = g.c;
+  key.P = g.P;
+  key.nsum = g.nsum;
+  key.BH = BH;
+  key.d = d;
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  int victim = -1;
+  for (int e = 0; e < kCacheSize; ++e) {
+    if (g_cache[e].valid && g_cache[e].key == key) {
+      g_cache[e].stamp = ++g_clock;
+      std::memcpy(out, g_cache[e].maps, sizeof(g_cache[e].maps));
+      return true;
+    }
+    // the first free slot, else the least recently used one
+    if (victim < 0 || (g_cache[victim].valid &&
+                       (!g_cache[e].valid || g_cache[e].stamp < g_cache[victim].stamp)))
+      victim = e;
+  }
+  if (!encode_views(out, base, is_f32, g, BH, d)) return false;
+  g_cache[victim].key = key;
+  std::memcpy(g_cache[victim].maps, out, sizeof(g_cache[victim].maps));
+  g_cache[victim].stamp = ++g_clock;
+  g_cache[victim].valid = true;
+  return true;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
 }
 
 }  // namespace st
