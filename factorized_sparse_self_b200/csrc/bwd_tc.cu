@@ -22,9 +22,12 @@
 //                    or dV (w = 1) at the end of a unit;
 //   warpgroup 2      warp 8 TMA producer (K, V per unit; Q, dO per query
 //                    tile into a 2-stage ring, with LSE and D by plain loads),
-//                    warp 9 TMEM owner and MMA issuer.
-// The MMA warp issues S, dP of the next tile before dV, dK, dQ of the current
-// one, so the exponentials overlap the tensor pipe. All waits are bounded.
+//                    warp 9 TMEM owner and MMA issuer, warp 10 reducer (TMA
+//                    reduce-adds of the staged dQ, dK, dV tiles, so that no
+//                    compute warp waits on a bulk copy).
+// The MMA warp issues S, dP of the next tile as soon as the compute warps hold
+// the current tile's in registers, ahead of dV, dK, dQ of the current tile,
+// so the exponentials overlap the tensor pipe. All waits are bounded.
 #include <math.h>
 
 #include <algorithm>
@@ -40,7 +43,7 @@ using namespace tc;
 constexpr int NS = 2;
 constexpr int kTileBytes = kTile * 64 * 2;  // 128 x 64 bf16 = 16 KB
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsCompute = 208, kRegsIssue = 88;  // launch: 168 per thread
+constexpr uint32_t kRegsCompute = 200, kRegsIssue = 104;  // launch: 168 per thread
 static_assert(256 * kRegsCompute + 128 * kRegsIssue == kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
@@ -62,7 +65,7 @@ struct SmemBwd {
   float l2[NS][kTile];           // LSE_i * log2(e) of the stage's query rows
   float dd[NS][kTile];           // D_i
   uint64_t kv_full, kv_done, full[NS], empty[NS];
-  uint64_t s_full, dp_full, ds_ready, pds_free, dq_full, dq_free, stg_full, stg_free;
+  uint64_t s_full, dp_full, sdp_free, ds_ready, pds_free, dq_full, dq_free, stg_full, stg_free;
   uint64_t acc_free, out_full, kvstg_free, fin;
   uint32_t tmem_base;
   int abort;
@@ -77,6 +80,19 @@ __device__ __forceinline__ void load_tile(void* dst, const CUtensorMap* maps, in
   } else {
     int r = tile / g.ptiles, pb = tile - r * g.ptiles;
     tma_load_4d(dst, &maps[VIEW_CLS], bar, 0, r, pb * kTile, bh);
+  }
+}
+
+// Prefetches a tile into L2 (the actual load follows when a ring stage frees).
+__device__ __forceinline__ void prefetch_tile(const CUtensorMap* maps, int view, const Geom& g,
+                                              int tile, int bh) {
+  if (view == VIEW_NAT) {
+    tma_prefetch_3d(&maps[VIEW_NAT], 0, tile * kTile, bh);
+  } else if (view == VIEW_SUM) {
+    tma_prefetch_4d(&maps[VIEW_SUM], 0, g.l - g.c, tile * (kTile / g.c), bh);
+  } else {
+    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+    tma_prefetch_4d(&maps[VIEW_CLS], 0, r, pb * kTile, bh);
   }
 }
 
@@ -169,6 +185,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     }
     mbar_init(&S.s_full, 1);
     mbar_init(&S.dp_full, 1);
+    mbar_init(&S.sdp_free, 256);
     mbar_init(&S.ds_ready, 256);
     mbar_init(&S.pds_free, 1);
     mbar_init(&S.dq_full, 1);
@@ -215,6 +232,11 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             mbar_arrive_expect_tx(&S.full[s], 2 * kTileBytes);
             load_tile(S.q[s], maps.q, x.it.qview, g, qe.qtile, x.bh, &S.full[s]);
             load_tile(S.dout[s], maps.dout, x.it.qview, g, qe.qtile, x.bh, &S.full[s]);
+            if (e + 2 < cnt) {  // two tiles ahead of the ring: into L2 now
+              const int pt = qents[x.it.qbeg + e + 2].qtile;
+              prefetch_tile(maps.q, x.it.qview, g, pt, x.bh);
+              prefetch_tile(maps.dout, x.it.qview, g, pt, x.bh);
+            }
           }
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
@@ -291,15 +313,19 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           if (ok) ok = issue_s_dp(gt);
           for (int e = 0; ok && e < cnt; ++e, ++gt) {
             const int s = gt % NS;
+            // S^T, dP^T of the next tile as soon as the compute warps hold this
+            // tile's in registers
+            if (e + 1 < cnt) {
+              if (!mbar_wait(&S.sdp_free, gt & 1, wait_ns, abort) || !issue_s_dp(gt + 1)) {
+                ok = false;
+                break;
+              }
+            }
             if (!mbar_wait(&S.ds_ready, gt & 1, wait_ns, abort)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            if (e + 1 < cnt && !issue_s_dp(gt + 1)) {
-              ok = false;
-              break;
-            }
             if (e == 0 && !mbar_wait(&S.acc_free, (n & 1) ^ 1, wait_ns, abort)) {
               ok = false;
               break;
@@ -317,6 +343,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
               mma_ss(tmem + kColDK,
                      sdesc(ds_addr + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
                      sdesc(q_addr + kk * 2048, 16384, 1024), idKM, (e > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&S.empty[s]);  // Q, dO of this stage are no longer read
             if (gt > 0 && !mbar_wait(&S.dq_free, (gt - 1) & 1, wait_ns, abort)) {
               ok = false;
               break;
@@ -329,7 +356,6 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
                      sdesc(k_addr + kk * 2048, 16384, 1024), idMM, kk > 0 ? 1u : 0u);
             mma_commit(&S.dq_full);
             mma_commit(&S.pds_free);
-            mma_commit(&S.empty[s]);
           }
           if (!ok) break;
           mma_commit(&S.kv_done);
@@ -339,6 +365,49 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         mma_commit(&S.fin);
         mbar_wait(&S.fin, 0, wait_ns, abort);
       }
+    } else if (warp == 10) {
+      // ---------------- reducer: TMA reduce-adds of the staged fp32 tiles ----------------
+      if (lane == 0) {
+        bool ok = true;
+        int gt = 0, n = 0;
+        int pv = 0, ptile = 0, pbh = 0;  // query tile of tile gt - 1
+        auto reduce_dq = [&](int t) -> bool {
+          if (!mbar_wait(&S.stg_full, t & 1, wait_ns, abort)) return false;
+          reduce_tile(maps.dq, pv, g, ptile, pbh, S.stage);
+          bulk_commit();
+          bulk_wait_read_all();
+          mbar_arrive(&S.stg_free);
+          return true;
+        };
+        for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+          const Unit x = unit_of(items, u, NH, B, H, nclasses);
+          if (x.bh < 0) continue;
+          const int cnt = x.it.qend - x.it.qbeg;
+          for (int e = 0; ok && e < cnt; ++e, ++gt) {
+            if (gt > 0 && !reduce_dq(gt - 1)) {
+              ok = false;
+              break;
+            }
+            pv = x.it.qview;
+            ptile = qents[x.it.qbeg + e].qtile;
+            pbh = x.bh;
+          }
+          if (!ok) break;
+          if (!mbar_wait(&S.out_full, n & 1, wait_ns, abort)) {
+            ok = false;
+            break;
+          }
+          reduce_tile(maps.dk, x.it.kview, g, x.it.ktile, x.bh, S.pt);
+          reduce_tile(maps.dv, x.it.kview, g, x.it.ktile, x.bh, S.dst);
+          bulk_commit();
+          bulk_wait_read_all();
+          mbar_arrive(&S.kvstg_free);
+          ++n;
+        }
+        if (ok && gt > 0 && !reduce_dq(gt - 1)) ok = false;
+        if (!ok) fail();
+        bulk_wait_all();
+      }
     }
   } else {
     regs_increase<kRegsCompute>();
@@ -347,13 +416,10 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     const int lg = warp & 3;
     const int row = lg * 32 + lane;              // key row (S^T, dP^T) / query row (dQ)
     const uint32_t tl = (uint32_t)(lg * 32) << 16;
-    const bool issuer = (warp == 0 && lane == 0);
     bool ok = true;
     const uint32_t pt_addr = smem_u32(S.pt), ds_addr = smem_u32(S.dst);
     const uint32_t st_addr = smem_u32(S.stage);
     int gt = 0, n = 0;
-    // query tile whose dQ is still in TMEM (drained after the next tile's dS)
-    int pend_view = 0, pend_tile = 0, pend_bh = 0;
 
     // dQ of tile t: TMEM -> registers -> fp32 staging -> TMA reduce-add
     auto drain_dq = [&](int t) -> bool {
@@ -373,13 +439,6 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
                      dq[ch * 4 + 2], dq[ch * 4 + 3]);
       fence_async_smem();
       mbar_arrive(&S.stg_full);
-      if (issuer) {
-        if (!mbar_wait(&S.stg_full, t & 1, wait_ns, abort)) return false;
-        reduce_tile(maps.dq, pend_view, g, pend_tile, pend_bh, S.stage);
-        bulk_commit();
-        bulk_wait_read_all();
-        mbar_arrive(&S.stg_free);
-      }
       return true;
     };
 
@@ -411,6 +470,8 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         tmem_ld32(tmem + tl + kColDP + wg * 64, reinterpret_cast<uint32_t*>(dp));
         tmem_ld32(tmem + tl + kColDP + wg * 64 + 32, reinterpret_cast<uint32_t*>(dp) + 32);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&S.sdp_free);  // S^T, dP^T of this tile may now be overwritten
         if (!full) {
 #pragma unroll
           for (int xk = 0; xk < 64; ++xk)
@@ -450,9 +511,6 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           ok = false;
           break;
         }
-        pend_view = it.qview;
-        pend_tile = qe.qtile;
-        pend_bh = x.bh;
       }
       if (!ok) break;
       // ---- end of unit: dK (warpgroup 0) or dV (warpgroup 1) -> reduce-add ----
@@ -477,22 +535,10 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
                        r[h * 32 + ch * 4 + 1], r[h * 32 + ch * 4 + 2], r[h * 32 + ch * 4 + 3]);
       fence_async_smem();
       mbar_arrive(&S.out_full);
-      if (issuer) {
-        if (!mbar_wait(&S.out_full, n & 1, wait_ns, abort)) {
-          ok = false;
-          break;
-        }
-        reduce_tile(maps.dk, it.kview, g, it.ktile, x.bh, S.pt);
-        reduce_tile(maps.dv, it.kview, g, it.ktile, x.bh, S.dst);
-        bulk_commit();
-        bulk_wait_read_all();
-        mbar_arrive(&S.kvstg_free);
-      }
       ++n;
     }
     if (ok && gt > 0 && !drain_dq(gt - 1)) ok = false;
     if (!ok) fail();
-    if (issuer) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();

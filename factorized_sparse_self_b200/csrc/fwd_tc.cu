@@ -11,9 +11,10 @@
 // A CTA walks a strided share of the work units (query tile x head, longest
 // first). Warp roles:
 //   warp 4       TMA producer: each unit's Q tile into one of two Q buffers
-//                (the next unit's Q loads while the current one computes),
-//                K and V tiles into a 2-stage ring (natural, summary or
-//                residue-class view);
+//                (the next unit's Q loads while the current one computes)
+//                and K tiles into a 2-stage ring released by the S MMA;
+//   warp 6       TMA producer: V tiles into a 2-stage ring released by PV
+//                (natural, summary or residue-class view for both);
 //   warp 5       TMEM owner and MMA issuer: S = Q K^T (M=128, N=128, K=64)
 //                into TMEM, then O += P V with P read from TMEM (A operand)
 //                and V from shared memory (MN-major);
@@ -54,8 +55,8 @@ struct SmemFwd {
   uint8_t q[2][kTileBytes];
   uint8_t k[NS][kTileBytes];
   uint8_t v[NS][kTileBytes];
-  uint64_t q_full[2], q_empty[2], kv_full[NS], kv_empty[NS];
-  uint64_t s_full, s_free, p_full, pv_done, o_full, o_free, fin;
+  uint64_t q_full[2], q_empty[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
+  uint64_t s_full, s_free, p_full, pv_done, o_free, fin;
   uint32_t tmem_base;
   int abort;
 };
@@ -69,6 +70,19 @@ __device__ __forceinline__ void load_tile(void* dst, const CUtensorMap* maps, in
   } else {
     int r = tile / g.ptiles, pb = tile - r * g.ptiles;
     tma_load_4d(dst, &maps[VIEW_CLS], bar, 0, r, pb * kTile, bh);
+  }
+}
+
+// Prefetches a tile into L2 (the actual load follows when a ring stage frees).
+__device__ __forceinline__ void prefetch_tile(const CUtensorMap* maps, int view, const Geom& g,
+                                              int tile, int bh) {
+  if (view == VIEW_NAT) {
+    tma_prefetch_3d(&maps[VIEW_NAT], 0, tile * kTile, bh);
+  } else if (view == VIEW_SUM) {
+    tma_prefetch_4d(&maps[VIEW_SUM], 0, g.l - g.c, tile * (kTile / g.c), bh);
+  } else {
+    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+    tma_prefetch_4d(&maps[VIEW_CLS], 0, r, pb * kTile, bh);
   }
 }
 
@@ -144,14 +158,15 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       mbar_init(&S.q_empty[b], 1);
     }
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&S.kv_full[s], 1);
-      mbar_init(&S.kv_empty[s], 1);
+      mbar_init(&S.k_full[s], 1);
+      mbar_init(&S.k_empty[s], 1);
+      mbar_init(&S.v_full[s], 1);
+      mbar_init(&S.v_empty[s], 1);
     }
     mbar_init(&S.s_full, 1);
     mbar_init(&S.s_free, 128);
     mbar_init(&S.p_full, 128);
     mbar_init(&S.pv_done, 1);
-    mbar_init(&S.o_full, 1);
     mbar_init(&S.o_free, 128);
     mbar_init(&S.fin, 1);
     S.abort = 0;
@@ -176,7 +191,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
   if (warp >= 4) {
     regs_decrease<kRegsIssue>();
   if (warp == 4) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer: Q and K ----------------
     if (lane == 0) {
       int kv_last[NS] = {-1, -1};
       int q_last[2] = {-1, -1};
@@ -196,15 +211,18 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         q_last[qb] = n;
         for (int e = x.it.kbeg; e < x.it.kend; ++e, ++gt) {
           const int s = gt % NS;
-          if (!mbar_wait(&S.kv_empty[s], ((gt / NS) & 1) ^ 1, wait_ns, abort)) {
+          if (!mbar_wait(&S.k_empty[s], ((gt / NS) & 1) ^ 1, wait_ns, abort)) {
             ok = false;
             break;
           }
           if (force_timeout && gt == 0) continue;  // test hook: this stage never fills
           const KeyEnt ke = keys[e];
-          mbar_arrive_expect_tx(&S.kv_full[s], 2 * kTileBytes);
-          load_tile(S.k[s], maps.k, ke.kview, g, ke.ktile, x.bh, &S.kv_full[s]);
-          load_tile(S.v[s], maps.v, ke.kview, g, ke.ktile, x.bh, &S.kv_full[s]);
+          mbar_arrive_expect_tx(&S.k_full[s], kTileBytes);
+          load_tile(S.k[s], maps.k, ke.kview, g, ke.ktile, x.bh, &S.k_full[s]);
+          if (e + 2 < x.it.kend) {
+            const KeyEnt kn = keys[e + 2];
+            prefetch_tile(maps.k, kn.kview, g, kn.ktile, x.bh);
+          }
           kv_last[s] = gt;
         }
         ++n;
@@ -215,7 +233,37 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         if (q_last[b] >= 0 && !mbar_wait(&S.q_full[b], (q_last[b] >> 1) & 1, wait_ns, abort))
           fail();
       for (int s = 0; s < NS; ++s)
-        if (kv_last[s] >= 0 && !mbar_wait(&S.kv_full[s], (kv_last[s] / NS) & 1, wait_ns, abort))
+        if (kv_last[s] >= 0 && !mbar_wait(&S.k_full[s], (kv_last[s] / NS) & 1, wait_ns, abort))
+          fail();
+    }
+  } else if (warp == 6) {
+    // ---------------- TMA producer: V (its own ring, freed by PV) ----------------
+    if (lane == 0) {
+      int v_last[NS] = {-1, -1};
+      int gt = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        const Unit x = unit_of(items, u, NH, B, H, nclasses);
+        if (x.bh < 0) continue;
+        for (int e = x.it.kbeg; e < x.it.kend; ++e, ++gt) {
+          const int s = gt % NS;
+          if (!mbar_wait(&S.v_empty[s], ((gt / NS) & 1) ^ 1, wait_ns, abort)) {
+            ok = false;
+            break;
+          }
+          const KeyEnt ke = keys[e];
+          mbar_arrive_expect_tx(&S.v_full[s], kTileBytes);
+          load_tile(S.v[s], maps.v, ke.kview, g, ke.ktile, x.bh, &S.v_full[s]);
+          if (e + 2 < x.it.kend) {  // two tiles ahead of the ring: into L2 now
+            const KeyEnt kn = keys[e + 2];
+            prefetch_tile(maps.v, kn.kview, g, kn.ktile, x.bh);
+          }
+          v_last[s] = gt;
+        }
+      }
+      if (!ok) fail();
+      for (int s = 0; s < NS; ++s)
+        if (v_last[s] >= 0 && !mbar_wait(&S.v_full[s], (v_last[s] / NS) & 1, wait_ns, abort))
           fail();
     }
   } else if (warp == 5) {
@@ -228,7 +276,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       // S of global tile g from Q buffer qb and K ring stage g % NS.
       auto issue_s = [&](int g, int qb) -> bool {
         const int s = g % NS;
-        if (!mbar_wait(&S.kv_full[s], (g / NS) & 1, wait_ns, abort)) return false;
+        if (!mbar_wait(&S.k_full[s], (g / NS) & 1, wait_ns, abort)) return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(S.q[qb]), k_addr = smem_u32(S.k[s]);
 #pragma unroll
@@ -236,6 +284,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           mma_ss(tmem + kColS, sdesc(q_addr + kk * 32, 16, 1024),
                  sdesc(k_addr + kk * 32, 16, 1024), idS, kk > 0);
         mma_commit(&S.s_full);
+        mma_commit(&S.k_empty[s]);
         return true;
       };
       // first unit at or after u with a valid head
@@ -302,6 +351,10 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
             ok = false;
             break;
           }
+          if (!mbar_wait(&S.v_full[s], (gt / NS) & 1, wait_ns, abort)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t v_addr = smem_u32(S.v[s]);
 #pragma unroll
@@ -309,11 +362,10 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
             mma_ts(tmem + kColO, tmem + kColP + kk * 8, sdesc(v_addr + kk * 2048, 16384, 1024),
                    idPV, (e > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&S.pv_done);
-          mma_commit(&S.kv_empty[s]);
+          mma_commit(&S.v_empty[s]);
         }
         if (!ok) break;
         mma_commit(&S.q_empty[qb]);
-        mma_commit(&S.o_full);
         ++n;
         u = un;
         cur = nx;
@@ -331,6 +383,63 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
     const uint32_t tl = (uint32_t)(lg * 32) << 16;
     bool ok = true;
     int gt = 0, n = 0;
+    // A unit's epilogue (O / l, merge, stores) runs inside the next unit's
+    // first tile: after that tile's exponentials, at the point where the last
+    // PV of the unit has to be complete anyway before P is overwritten.
+    struct Pending {
+      int i, bh, cnt, merge;
+      float m, l;
+    };
+    Pending pend = {-1, 0, 0, 0, 0.f, 0.f};
+    bool pending = false;
+    auto epilogue = [&](const Pending& pe) {
+      float o[64];
+#pragma unroll
+      for (int xk = 0; xk < 64; ++xk) o[xk] = 0.f;
+      if (pe.cnt > 0) {
+        tmem_ld32(tmem + tl + kColO, reinterpret_cast<uint32_t*>(o));
+        tmem_ld32(tmem + tl + kColO + 32, reinterpret_cast<uint32_t*>(o) + 32);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(&S.o_free);
+      if (pe.i < 0) return;
+      const float inv = (pe.l > 0.f) ? 1.f / pe.l : 0.f;
+      float L = (pe.l > 0.f) ? (pe.m + __log2f(pe.l)) * 0.69314718055994531f : -INFINITY;
+#pragma unroll
+      for (int xk = 0; xk < 64; ++xk) o[xk] *= inv;
+      const size_t rowoff = ((size_t)pe.bh * g.T + pe.i) * 64;
+      uint4* dst = reinterpret_cast<uint4*>(out + rowoff);
+      if (pe.merge) {
+        const float Lp = lse[(size_t)pe.bh * g.T + pe.i];
+        const float mx2 = fmaxf(Lp, L);
+        float wp = 0.f, wc = 0.f;
+        if (mx2 != -INFINITY) {
+          const float Ln = mx2 + __logf(__expf(Lp - mx2) + __expf(L - mx2));
+          wp = __expf(Lp - Ln);
+          wc = __expf(L - Ln);
+          L = Ln;
+        }
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint4 w = dst[ch];
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ws[q2]));
+            o[ch * 8 + 2 * q2] = fmaf(wp, f.x, wc * o[ch * 8 + 2 * q2]);
+            o[ch * 8 + 2 * q2 + 1] = fmaf(wp, f.y, wc * o[ch * 8 + 2 * q2 + 1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        dst[ch] = make_uint4(pack_bf16(o[ch * 8 + 0], o[ch * 8 + 1]),
+                             pack_bf16(o[ch * 8 + 2], o[ch * 8 + 3]),
+                             pack_bf16(o[ch * 8 + 4], o[ch * 8 + 5]),
+                             pack_bf16(o[ch * 8 + 6], o[ch * 8 + 7]));
+      lse[(size_t)pe.bh * g.T + pe.i] = L;
+    };
     for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
       const Unit x = unit_of(items, u, NH, B, H, nclasses);
       if (x.bh < 0) continue;
@@ -338,6 +447,19 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       const int bh = x.bh;
       const int i = view_pos(g, it.qview, it.qtile, row);
       const int cnt = it.kend - it.kbeg;
+      if (cnt == 0) {
+        if (pending) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&S.pv_done, (gt - 1) & 1, wait_ns, abort));
+          if (!ok) break;
+          tc_fence_after();
+          epilogue(pend);
+          pending = false;
+        }
+        const Pending z = {i, bh, 0, (int)it.merge, -INFINITY, 0.f};
+        epilogue(z);
+        ++n;
+        continue;
+      }
       float m_run = -INFINITY, l_run = 0.f;
       for (int e = 0; e < cnt; ++e, ++gt) {
         const KeyEnt ke = keys[it.kbeg + e];
@@ -380,11 +502,31 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           m_run = m_new;
         }
         const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+        // exponentials: one packed FMA forms two exponents, masked entries are
+        // -inf and give exactly 0; four pairs of partial sums break the add chain
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        const float nmu = -mu;
+        uint32_t pk[64];
+#pragma unroll
+        for (int xk = 0; xk < 128; xk += 2) {
+          float a0, a1;
+          ffma2(a0, a1, s[xk], s[xk + 1], scale_log2, scale_log2, nmu, nmu);
+          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+          const int j = (xk >> 1) & 3;
+          fadd2(sa[j], sb[j], sa[j], sb[j], p0, p1);
+          pk[xk >> 1] = pack_bf16(p0, p1);
+        }
+        l_run = l_run * alpha + (((sa[0] + sb[0]) + (sa[1] + sb[1])) +
+                                 ((sa[2] + sb[2]) + (sa[3] + sb[3])));
         if (gt > 0) {
           // PV of the previous tile is done: P may be overwritten, O is stable
           ok = __all_sync(0xffffffffu, mbar_wait(&S.pv_done, (gt - 1) & 1, wait_ns, abort));
           if (!ok) break;
           tc_fence_after();
+        }
+        if (e == 0 && pending) {
+          epilogue(pend);
+          pending = false;
         }
         if (__any_sync(0xffffffffu, rescale_o)) {
           const float a = rescale_o ? alpha : 1.f;
@@ -398,80 +540,23 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
             tmem_st8(tmem + tl + kColO + c8 * 8, o);
           }
         }
-        // exp pass: one packed FMA forms two exponents, masked entries are -inf
-        // and give exactly 0; four pairs of partial sums break the add chain.
-        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-        const float nmu = -mu;
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          uint32_t pk[8];  // 16 keys at a time keeps the live set near S itself
-#pragma unroll
-          for (int xk = 0; xk < 16; xk += 2) {
-            float a0, a1;
-            ffma2(a0, a1, s[h * 16 + xk], s[h * 16 + xk + 1], scale_log2, scale_log2, nmu, nmu);
-            const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
-            const int j = (xk >> 1) & 3;
-            fadd2(sa[j], sb[j], sa[j], sb[j], p0, p1);
-            pk[xk >> 1] = pack_bf16(p0, p1);
-          }
-          tmem_st8(tmem + tl + kColP + h * 8, pk);
-        }
-        l_run = l_run * alpha + (((sa[0] + sb[0]) + (sa[1] + sb[1])) +
-                                 ((sa[2] + sb[2]) + (sa[3] + sb[3])));
+        tmem_st32(tmem + tl + kColP, pk);
+        tmem_st32(tmem + tl + kColP + 32, pk + 32);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&S.p_full);
       }
       if (!ok) break;
-      // ---- epilogue of the unit ----
-      ok = __all_sync(0xffffffffu, mbar_wait(&S.o_full, n & 1, wait_ns, abort));
-      if (!ok) break;
-      tc_fence_after();
-      float o[64];
-      if (cnt > 0) {
-        tmem_ld32(tmem + tl + kColO, reinterpret_cast<uint32_t*>(o));
-        tmem_ld32(tmem + tl + kColO + 32, reinterpret_cast<uint32_t*>(o) + 32);
-        tmem_wait_ld();
-      }
-      tc_fence_before();
-      mbar_arrive(&S.o_free);
+      pend = {i, bh, cnt, (int)it.merge, m_run, l_run};
+      pending = true;
       ++n;
-      if (i < 0) continue;
-      const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-      float L = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
-#pragma unroll
-      for (int xk = 0; xk < 64; ++xk) o[xk] = (cnt > 0) ? o[xk] * inv : 0.f;
-      const size_t rowoff = ((size_t)bh * g.T + i) * 64;
-      uint4* dst = reinterpret_cast<uint4*>(out + rowoff);
-      if (it.merge) {
-        const float Lp = lse[(size_t)bh * g.T + i];
-        const float mx2 = fmaxf(Lp, L);
-        float wp = 0.f, wc = 0.f;
-        if (mx2 != -INFINITY) {
-          const float Ln = mx2 + __logf(__expf(Lp - mx2) + __expf(L - mx2));
-          wp = __expf(Lp - Ln);
-          wc = __expf(L - Ln);
-          L = Ln;
-        }
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint4 w = dst[ch];
-          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int q2 = 0; q2 < 4; ++q2) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ws[q2]));
-            o[ch * 8 + 2 * q2] = fmaf(wp, f.x, wc * o[ch * 8 + 2 * q2]);
-            o[ch * 8 + 2 * q2 + 1] = fmaf(wp, f.y, wc * o[ch * 8 + 2 * q2 + 1]);
-          }
-        }
+    }
+    if (ok && pending) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&S.pv_done, (gt - 1) & 1, wait_ns, abort));
+      if (ok) {
+        tc_fence_after();
+        epilogue(pend);
       }
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        dst[ch] = make_uint4(pack_bf16(o[ch * 8 + 0], o[ch * 8 + 1]),
-                             pack_bf16(o[ch * 8 + 2], o[ch * 8 + 3]),
-                             pack_bf16(o[ch * 8 + 4], o[ch * 8 + 5]),
-                             pack_bf16(o[ch * 8 + 6], o[ch * 8 + 7]));
-      lse[(size_t)bh * g.T + i] = L;
     }
     if (!ok) fail();
   }
