@@ -9,10 +9,12 @@
 //   dS^T = P^T (dP^T - D_i),      D_i = dO_i . O_i (prologue kernel)
 //   dV  += P^T dO                 (M=128, N=64, K=128)
 //   dK  += dS^T Q
-//   dQ_i = dS K  -> TMA reduce-add into the fp32 dQ accumulator
+//   dQ_i = dS K
 // dV and dK stay in TMEM for a whole work unit (a key tile, or a chunk of a
-// long key column) and are reduce-added into fp32 accumulators at its end; an
-// epilogue kernel applies the scale and rounds to bf16.
+// long key column). A gradient tile whose rows no other unit (for dK, dV) or
+// pair (for dQ) touches is scaled, rounded to bf16 and TMA-stored straight
+// into the output; every other tile is TMA reduce-added into an fp32
+// accumulator, which a later kernel scales and rounds.
 //
 // Persistent CTAs, one per SM, each walking a strided share of the work units
 // (longest first). Warpgroup roles:
@@ -52,6 +54,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct BwdMaps {
   CUtensorMap q[3], k[3], v[3], dout[3];  // bf16, indexed by View
   CUtensorMap dq[3], dk[3], dv[3];        // fp32 accumulators, 32-float boxes
+  CUtensorMap dqo[3], dko[3], dvo[3];     // bf16 outputs (direct tiles)
 };
 
 struct SmemBwd {
@@ -61,7 +64,7 @@ struct SmemBwd {
   uint8_t dout[NS][kTileBytes];
   uint8_t pt[2 * kTileBytes];    // P^T (keys x queries), two 64-query K-blocks
   uint8_t dst[2 * kTileBytes];   // dS^T, same layout
-  uint8_t stage[2 * kTileBytes]; // fp32 dQ tile for the reduce: two 32-column halves
+  uint8_t stage[2 * kTileBytes]; // dQ tile: fp32 in two 32-column halves, or bf16
   float l2[NS][kTile];           // LSE_i * log2(e) of the stage's query rows
   float dd[NS][kTile];           // D_i
   uint64_t kv_full, kv_done, full[NS], empty[NS];
@@ -111,6 +114,26 @@ __device__ __forceinline__ void reduce_tile(const CUtensorMap* maps, int view, c
       tma_reduce_add_4d(&maps[VIEW_CLS], s, h * 32, r, pb * kTile, bh);
     }
   }
+}
+
+// Stores a 128-row bf16 tile (coordinates are never negative).
+__device__ __forceinline__ void store_tile(const CUtensorMap* maps, int view, const Geom& g,
+                                           int tile, int bh, const uint8_t* src) {
+  if (view == VIEW_NAT) {
+    tma_store_3d(&maps[VIEW_NAT], src, 0, tile * kTile, bh);
+  } else if (view == VIEW_SUM) {
+    tma_store_4d(&maps[VIEW_SUM], src, 0, g.l - g.c, tile * (kTile / g.c), bh);
+  } else {
+    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+    tma_store_4d(&maps[VIEW_CLS], src, 0, r, pb * kTile, bh);
+  }
+}
+
+// Eight fp32 values (bit patterns), times s, as four packed bf16 pairs.
+__device__ __forceinline__ void round8(const uint32_t* v, float s, uint32_t w[4]) {
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+    w[x] = pack_bf16(__uint_as_float(v[2 * x]) * s, __uint_as_float(v[2 * x + 1]) * s);
 }
 
 // Live query columns [lo, hi) of a query tile for the key at natural
@@ -168,7 +191,7 @@ __device__ __forceinline__ Unit unit_of(const BwdItem* items, int u, int NH, int
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __restrict__ items,
               int n_units, int NH, const QEnt* __restrict__ qents, int B, int H, int nclasses,
-              float scale_log2, const float* __restrict__ lse, const float* __restrict__ Dg,
+              float scale, float scale_log2, const float* __restrict__ lse, const float* __restrict__ Dg,
               int* status, uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   SmemBwd& S = *reinterpret_cast<SmemBwd*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -370,10 +393,13 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       if (lane == 0) {
         bool ok = true;
         int gt = 0, n = 0;
-        int pv = 0, ptile = 0, pbh = 0;  // query tile of tile gt - 1
+        int pv = 0, ptile = 0, pbh = 0, pdirect = 0;  // query tile of tile gt - 1
         auto reduce_dq = [&](int t) -> bool {
           if (!mbar_wait(&S.stg_full, t & 1, wait_ns, abort)) return false;
-          reduce_tile(maps.dq, pv, g, ptile, pbh, S.stage);
+          if (pdirect)
+            store_tile(maps.dqo, pv, g, ptile, pbh, S.stage);
+          else
+            reduce_tile(maps.dq, pv, g, ptile, pbh, S.stage);
           bulk_commit();
           bulk_wait_read_all();
           mbar_arrive(&S.stg_free);
@@ -388,8 +414,10 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
               ok = false;
               break;
             }
+            const QEnt qe = qents[x.it.qbeg + e];
             pv = x.it.qview;
-            ptile = qents[x.it.qbeg + e].qtile;
+            ptile = qe.qtile;
+            pdirect = qe.q_direct;
             pbh = x.bh;
           }
           if (!ok) break;
@@ -397,8 +425,13 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             ok = false;
             break;
           }
-          reduce_tile(maps.dk, x.it.kview, g, x.it.ktile, x.bh, S.pt);
-          reduce_tile(maps.dv, x.it.kview, g, x.it.ktile, x.bh, S.dst);
+          if (x.it.kv_direct) {
+            store_tile(maps.dko, x.it.kview, g, x.it.ktile, x.bh, S.pt);
+            store_tile(maps.dvo, x.it.kview, g, x.it.ktile, x.bh, S.dst);
+          } else {
+            reduce_tile(maps.dk, x.it.kview, g, x.it.ktile, x.bh, S.pt);
+            reduce_tile(maps.dv, x.it.kview, g, x.it.ktile, x.bh, S.dst);
+          }
           bulk_commit();
           bulk_wait_read_all();
           mbar_arrive(&S.kvstg_free);
@@ -420,9 +453,11 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     const uint32_t pt_addr = smem_u32(S.pt), ds_addr = smem_u32(S.dst);
     const uint32_t st_addr = smem_u32(S.stage);
     int gt = 0, n = 0;
+    int pend_direct = 0;  // q_direct of the tile whose dQ is pending
 
-    // dQ of tile t: TMEM -> registers -> fp32 staging -> TMA reduce-add
-    auto drain_dq = [&](int t) -> bool {
+    // dQ of tile t: TMEM -> registers -> staging (fp32 for the reduce-add, or
+    // scaled bf16 for the direct store)
+    auto drain_dq = [&](int t, int direct) -> bool {
       bool w = mbar_wait(&S.dq_full, t & 1, wait_ns, abort);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
@@ -433,10 +468,19 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       mbar_arrive(&S.dq_free);
       w = mbar_wait(&S.stg_free, (t & 1) ^ 1, wait_ns, abort);
       if (!__all_sync(0xffffffffu, w)) return false;
+      if (direct) {
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        st_shared_v4(st_addr + wg * kTileBytes + swz128(row, ch), dq[ch * 4 + 0], dq[ch * 4 + 1],
-                     dq[ch * 4 + 2], dq[ch * 4 + 3]);
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t o4[4];
+          round8(dq + ch * 8, scale, o4);
+          st_shared_v4(st_addr + swz128(row, wg * 4 + ch), o4[0], o4[1], o4[2], o4[3]);
+        }
+      } else {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          st_shared_v4(st_addr + wg * kTileBytes + swz128(row, ch), dq[ch * 4 + 0],
+                       dq[ch * 4 + 1], dq[ch * 4 + 2], dq[ch * 4 + 3]);
+      }
       fence_async_smem();
       mbar_arrive(&S.stg_full);
       return true;
@@ -507,10 +551,11 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(&S.ds_ready);
-        if (gt > 0 && !drain_dq(gt - 1)) {
+        if (gt > 0 && !drain_dq(gt - 1, pend_direct)) {
           ok = false;
           break;
         }
+        pend_direct = qe.q_direct;
       }
       if (!ok) break;
       // ---- end of unit: dK (warpgroup 0) or dV (warpgroup 1) -> reduce-add ----
@@ -527,17 +572,28 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       tc_fence_before();
       mbar_arrive(&S.acc_free);
       const uint32_t dst = wg ? ds_addr : pt_addr;
+      if (it.kv_direct) {
+        const float sc = wg ? 1.f : scale;  // dK carries the softmax scale, dV none
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t o4[4];
+          round8(r + ch * 8, sc, o4);
+          st_shared_v4(dst + swz128(row, ch), o4[0], o4[1], o4[2], o4[3]);
+        }
+      } else {
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          st_shared_v4(dst + h * kTileBytes + swz128(row, ch), r[h * 32 + ch * 4 + 0],
-                       r[h * 32 + ch * 4 + 1], r[h * 32 + ch * 4 + 2], r[h * 32 + ch * 4 + 3]);
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            st_shared_v4(dst + h * kTileBytes + swz128(row, ch), r[h * 32 + ch * 4 + 0],
+                         r[h * 32 + ch * 4 + 1], r[h * 32 + ch * 4 + 2],
+                         r[h * 32 + ch * 4 + 3]);
+      }
       fence_async_smem();
       mbar_arrive(&S.out_full);
       ++n;
     }
-    if (ok && gt > 0 && !drain_dq(gt - 1)) ok = false;
+    if (ok && gt > 0 && !drain_dq(gt - 1, pend_direct)) ok = false;
     if (!ok) fail();
   }
   tc_fence_before();
@@ -549,7 +605,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
 
 cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, const float* lse,
                    const void* dout, const float* D, float* dq_acc, float* dk_acc,
-                   float* dv_acc) {
+                   float* dv_acc, void* dq, void* dk, void* dv) {
   const st_layout* L = c.L;
   const int BH = c.B * c.H;
   if (L->dev.n_bwd_items == 0) return cudaSuccess;
@@ -560,7 +616,10 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, c
       !make_view_maps(maps.dout, dout, false, L->geom, BH, c.d) ||
       !make_view_maps(maps.dq, dq_acc, true, L->geom, BH, c.d) ||
       !make_view_maps(maps.dk, dk_acc, true, L->geom, BH, c.d) ||
-      !make_view_maps(maps.dv, dv_acc, true, L->geom, BH, c.d))
+      !make_view_maps(maps.dv, dv_acc, true, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dqo, dq, false, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dko, dk, false, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dvo, dv, false, L->geom, BH, c.d))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(SmemBwd) + 1024;
   static bool attr_set[64] = {false};
@@ -581,7 +640,8 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, c
   record_begin(c);
   bwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
       maps, L->geom, (const BwdItem*)L->dev.bwd_items, (int)units, NH,
-      (const QEnt*)L->dev.q_ents, c.B, c.H, c.nclasses, c.scale * kLog2e, lse, D, c.status,
+      (const QEnt*)L->dev.q_ents, c.B, c.H, c.nclasses, c.scale, c.scale * kLog2e, lse, D,
+      c.status,
       c.wait_ns);
   err = cudaGetLastError();
   record_end(c);

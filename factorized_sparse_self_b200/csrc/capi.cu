@@ -61,6 +61,8 @@ void free_device(st_layout* L) {
   cudaFree(L->dev.key_ents);
   cudaFree(L->dev.bwd_items);
   cudaFree(L->dev.q_ents);
+  for (int hc = 0; hc < 2; ++hc)
+    for (int k = 0; k < N_ROWLISTS; ++k) cudaFree(L->dev.rows[hc][k]);
   if (prev >= 0) cudaSetDevice(prev);
   L->on_device = false;
 }
@@ -171,6 +173,11 @@ st_status st_pattern_layout(const st_pattern_desc* desc, st_layout** out, void* 
   if (e == cudaSuccess) e = upload(&L->dev.bwd_items, L->bwd_items, cs);
   if (e == cudaSuccess) e = upload(&L->dev.q_ents, L->q_ents, cs);
   L->dev.n_bwd_items = (int32_t)L->bwd_items.size();
+  for (int hc = 0; hc < (int)L->hcs.size() && e == cudaSuccess; ++hc)
+    for (int k = 0; k < N_ROWLISTS && e == cudaSuccess; ++k) {
+      e = upload(&L->dev.rows[hc][k], L->rows[hc][k], cs);
+      L->dev.n_rows[hc][k] = (int32_t)L->rows[hc][k].size();
+    }
   if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
   if (e != cudaSuccess) {
     free_device(L);
@@ -317,14 +324,15 @@ st_status st_sparse_attn_bwd(const st_layout* L, st_dtype dtype, int32_t B, int3
     float* acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
                                           round256(rows * sizeof(float)));
     const size_t stride = round256(elems * sizeof(float)) / sizeof(float);
-    // the three accumulators must be back to back for the epilogue
-    if (stride != elems) return ST_ERR_UNSUPPORTED;
-    e = bwd_prologue(c, o, dout, Dv, acc, 3 * elems);
+    float* dq_acc = acc;
+    float* dk_acc = acc + stride;
+    float* dv_acc = acc + 2 * stride;
+    e = bwd_prep(c, o, dout, Dv, dq_acc, dk_acc, dv_acc, dq, dk, dv);
     Call cm = c;
     arm(cm, 1);
     if (e == cudaSuccess)
-      e = tc_bwd(cm, q, k, v, lse, dout, Dv, acc, acc + stride, acc + 2 * stride);
-    if (e == cudaSuccess) e = bwd_epilogue(c, acc, dq, dk, dv, elems);
+      e = tc_bwd(cm, q, k, v, lse, dout, Dv, dq_acc, dk_acc, dv_acc, dq, dk, dv);
+    if (e == cudaSuccess) e = bwd_finish(c, dq_acc, dk_acc, dv_acc, dq, dk, dv);
   }
   return e == cudaSuccess ? ST_OK : ST_ERR_CUDA;
 }

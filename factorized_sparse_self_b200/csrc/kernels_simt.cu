@@ -1,4 +1,5 @@
-// Exact-fp32 path on CUDA cores, plus the backward prologue and epilogue.
+// Exact-fp32 path on CUDA cores, plus the backward prologue (fp32) and the
+// prep / finish kernels around the bf16 tensor-core backward.
 //
 // The fp32 kernels walk the same schedule as the tensor-core kernels (work
 // items of 128-row query or key tiles, each with its live tiles) and test
@@ -11,6 +12,8 @@
 // "Sparse attention as an unnormalized form". Backward with the attention
 // matrix recomputed from LSE: milestone page, "Recomputation".
 #include <math.h>
+
+#include <algorithm>
 
 #include "device_common.cuh"
 #include "launch.h"
@@ -270,23 +273,117 @@ __global__ void prologue_kernel(const E* __restrict__ o, const E* __restrict__ d
     acc[t] = z;
 }
 
-// Rounds the fp32 accumulators (dQ, dK, dV back to back) into bf16 outputs;
-// dQ and dK are scaled here because the tensor-core kernel accumulates dS K
-// and dS^T Q unscaled.
-__global__ void epilogue_kernel(const float4* __restrict__ acc, __nv_bfloat162* __restrict__ dq,
-                                __nv_bfloat162* __restrict__ dk, __nv_bfloat162* __restrict__ dv,
-                                size_t vec, float scale) {
-  for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < vec;
-       t += gridDim.x * (size_t)blockDim.x) {
-    float4 a = acc[t], b = acc[vec + t], c = acc[2 * vec + t];
-    a.x *= scale; a.y *= scale; a.z *= scale; a.w *= scale;
-    b.x *= scale; b.y *= scale; b.z *= scale; b.w *= scale;
-    dq[2 * t] = __floats2bfloat162_rn(a.x, a.y);
-    dq[2 * t + 1] = __floats2bfloat162_rn(a.z, a.w);
-    dk[2 * t] = __floats2bfloat162_rn(b.x, b.y);
-    dk[2 * t + 1] = __floats2bfloat162_rn(b.z, b.w);
-    dv[2 * t] = __floats2bfloat162_rn(c.x, c.y);
-    dv[2 * t + 1] = __floats2bfloat162_rn(c.z, c.w);
+struct RowSet {
+  const int32_t* rows[2][N_ROWLISTS];
+  int32_t n[2][N_ROWLISTS];
+};
+
+// Row list k of head class hc, picked without dynamic indexing of the
+// parameter (which would copy it to local memory).
+__device__ __forceinline__ const int32_t* rows_of(const RowSet& rs, int hc, int k, int& n) {
+  n = hc ? rs.n[1][k] : rs.n[0][k];
+  return hc ? rs.rows[1][k] : rs.rows[0][k];
+}
+
+RowSet row_set_of(const st_layout* L) {
+  RowSet r;
+  for (int hc = 0; hc < 2; ++hc)
+    for (int k = 0; k < N_ROWLISTS; ++k) {
+      r.rows[hc][k] = (const int32_t*)L->dev.rows[hc][k];
+      r.n[hc][k] = L->dev.n_rows[hc][k];
+    }
+  return r;
+}
+
+// Grid (x, B*H); d = 64 bf16 rows of 128 bytes.
+__global__ void bwd_prep_kernel(const __nv_bfloat162* __restrict__ o,
+                                const __nv_bfloat162* __restrict__ dout, float* __restrict__ Dv,
+                                int T, int H, int nclasses, RowSet rs, float4* __restrict__ dq_acc,
+                                float4* __restrict__ dk_acc, float4* __restrict__ dv_acc,
+                                uint4* __restrict__ dq, uint4* __restrict__ dk,
+                                uint4* __restrict__ dv) {
+  const int bh = blockIdx.y;
+  const int hc = (nclasses == 2) ? ((bh % H) & 1) : 0;
+  const size_t rb = (size_t)bh * T;
+  const int lane = threadIdx.x & 31;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int r = warp; r < T; r += nwarps) {
+    const float2 a = __bfloat1622float2(o[(rb + r) * 32 + lane]);
+    const float2 b = __bfloat1622float2(dout[(rb + r) * 32 + lane]);
+    float sacc = fmaf(a.x, b.x, a.y * b.y);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, off);
+    if (lane == 0) Dv[rb + r] = sacc;
+  }
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int stride = gridDim.x * blockDim.x;
+  const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  const uint4 zu = make_uint4(0u, 0u, 0u, 0u);
+  {
+    int nr;
+    const int32_t* rows = rows_of(rs, hc, ROWS_Q_ACC, nr);
+    for (int64_t x = tid; x < (int64_t)nr * 16; x += stride)
+      dq_acc[(rb + rows[x >> 4]) * 16 + (x & 15)] = z4;
+  }
+  {
+    int nr;
+    const int32_t* rows = rows_of(rs, hc, ROWS_K_ACC, nr);
+    for (int64_t x = tid; x < (int64_t)nr * 16; x += stride) {
+      const size_t e = (rb + rows[x >> 4]) * 16 + (x & 15);
+      dk_acc[e] = z4;
+      dv_acc[e] = z4;
+    }
+  }
+  {
+    int nr;
+    const int32_t* rows = rows_of(rs, hc, ROWS_Q_ZERO, nr);
+    for (int64_t x = tid; x < (int64_t)nr * 8; x += stride)
+      dq[(rb + rows[x >> 3]) * 8 + (x & 7)] = zu;
+  }
+  {
+    int nr;
+    const int32_t* rows = rows_of(rs, hc, ROWS_K_ZERO, nr);
+    for (int64_t x = tid; x < (int64_t)nr * 8; x += stride) {
+      const size_t e = (rb + rows[x >> 3]) * 8 + (x & 7);
+      dk[e] = zu;
+      dv[e] = zu;
+    }
+  }
+}
+
+__device__ __forceinline__ uint2 round4(float4 a, float s) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a.x * s, a.y * s);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(a.z * s, a.w * s);
+  return make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+}
+
+__global__ void bwd_finish_kernel(const float4* __restrict__ dq_acc,
+                                  const float4* __restrict__ dk_acc,
+                                  const float4* __restrict__ dv_acc, int T, int H, int nclasses,
+                                  RowSet rs, float scale, uint2* __restrict__ dq,
+                                  uint2* __restrict__ dk, uint2* __restrict__ dv) {
+  const int bh = blockIdx.y;
+  const int hc = (nclasses == 2) ? ((bh % H) & 1) : 0;
+  const size_t rb = (size_t)bh * T;
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int stride = gridDim.x * blockDim.x;
+  {
+    int nr;
+    const int32_t* rows = rows_of(rs, hc, ROWS_Q_ACC, nr);
+    for (int64_t x = tid; x < (int64_t)nr * 16; x += stride) {
+      const size_t e = (rb + rows[x >> 4]) * 16 + (x & 15);
+      dq[e] = round4(dq_acc[e], scale);
+    }
+  }
+  {
+    int nr;
+    const int32_t* rows = rows_of(rs, hc, ROWS_K_ACC, nr);
+    for (int64_t x = tid; x < (int64_t)nr * 16; x += stride) {
+      const size_t e = (rb + rows[x >> 4]) * 16 + (x & 15);
+      dk[e] = round4(dk_acc[e], scale);
+      dv[e] = round4(dv_acc[e], 1.f);
+    }
   }
 }
 
@@ -398,13 +495,30 @@ cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* 
   return cudaGetLastError();
 }
 
-cudaError_t bwd_epilogue(const Call& c, const float* acc, void* dq, void* dk, void* dv,
-                         size_t elems) {
-  size_t vec = elems / 4;
-  int threads = 256;
-  epilogue_kernel<<<grid_cap(vec, threads), threads, 0, c.stream>>>(
-      (const float4*)acc, (__nv_bfloat162*)dq, (__nv_bfloat162*)dk, (__nv_bfloat162*)dv, vec,
-      c.scale);
+cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* Dv, float* dq_acc,
+                     float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv) {
+  const int T = c.L->geom.T;
+  const int bx = std::max(1, std::min(64, (T * 32 + 255) / 256));
+  dim3 grid(bx, c.B * c.H);
+  bwd_prep_kernel<<<grid, 256, 0, c.stream>>>(
+      (const __nv_bfloat162*)o, (const __nv_bfloat162*)dout, Dv, T, c.H, c.nclasses,
+      row_set_of(c.L), (float4*)dq_acc, (float4*)dk_acc, (float4*)dv_acc, (uint4*)dq, (uint4*)dk,
+      (uint4*)dv);
+  return cudaGetLastError();
+}
+
+cudaError_t bwd_finish(const Call& c, const float* dq_acc, const float* dk_acc,
+                       const float* dv_acc, void* dq, void* dk, void* dv) {
+  const st_layout* L = c.L;
+  int most = 0;
+  for (int hc = 0; hc < (int)L->hcs.size(); ++hc)
+    most = std::max(most, std::max(L->dev.n_rows[hc][ROWS_Q_ACC], L->dev.n_rows[hc][ROWS_K_ACC]));
+  if (most == 0) return cudaSuccess;  // every row was written directly
+  const int bx = std::max(1, std::min(64, (most * 16 + 255) / 256));
+  dim3 grid(bx, c.B * c.H);
+  bwd_finish_kernel<<<grid, 256, 0, c.stream>>>(
+      (const float4*)dq_acc, (const float4*)dk_acc, (const float4*)dv_acc, L->geom.T, c.H,
+      c.nclasses, row_set_of(L), c.scale, (uint2*)dq, (uint2*)dk, (uint2*)dv);
   return cudaGetLastError();
 }
 

@@ -38,19 +38,26 @@ cudaError_t simt_bwd(const Call& c, const void* q, const void* k, const void* v,
                      const float* lse, const void* dout, const float* D, float* dq_acc,
                      float* dk_acc, float* dv_acc);
 
-// Backward prologue (D_i = dout_i . O_i, zero the fp32 accumulators) and,
-// for bf16, the epilogue that rounds the accumulators into dq, dk, dv.
+// fp32 backward prologue: D_i = dout_i . O_i (and zeroes acc_elems floats).
 cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* D, float* acc,
                          size_t acc_elems);
-cudaError_t bwd_epilogue(const Call& c, const float* acc, void* dq, void* dk, void* dv,
-                         size_t elems);
+
+// bf16 backward, around the tensor-core kernel: bwd_prep writes D for every
+// row, zeroes the fp32 accumulator rows that collect several contributions and
+// zero-fills the output rows nobody writes; bwd_finish rounds the accumulated
+// rows into dq, dk, dv (scale applied to dQ and dK). Rows that a single
+// backward unit produces are written by the tensor-core kernel itself.
+cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* D, float* dq_acc,
+                     float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv);
+cudaError_t bwd_finish(const Call& c, const float* dq_acc, const float* dk_acc,
+                       const float* dv_acc, void* dq, void* dk, void* dv);
 
 // Tensor-core path (tcgen05 + TMA): bf16, d = 64.
 cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, void* o,
                    float* lse, int force_timeout);
 cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v,
                    const float* lse, const void* dout, const float* D, float* dq_acc,
-                   float* dk_acc, float* dv_acc);
+                   float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv);
 
 }  // namespace st
 

@@ -196,6 +196,71 @@ void build_segment(const SegDef& d, const Geom& g, Segment& seg, int64_t& nnz) {
   flush();
 }
 
+// Natural positions of the valid rows of tile `tile` in view v.
+void tile_rows(uint8_t v, const Geom& g, int32_t tile, std::vector<int32_t>& out) {
+  out.clear();
+  for (int k = 0; k < kTile; ++k) {
+    if (v == VIEW_NAT) {
+      const i64 t = (i64)tile * kTile + k;
+      if (t < g.T) out.push_back((int32_t)t);
+    } else if (v == VIEW_SUM) {
+      const i64 sg = (i64)tile * kTile + k;
+      if (sg < g.nsum) out.push_back((int32_t)((sg / g.c) * g.l + (g.l - g.c) + sg % g.c));
+    } else {
+      const i64 r = tile / g.ptiles, p = (i64)(tile - r * g.ptiles) * kTile + k;
+      if (p < g.P) out.push_back((int32_t)(p * g.l + r));
+    }
+  }
+}
+
+// Who writes each gradient row (bf16 path). A backward unit writes dK, dV of
+// its whole key tile, a (unit, query tile) pair writes dQ of the query tile.
+// A tile whose rows all have exactly one writer is written directly in bf16
+// by that writer; rows with several writers go through fp32 accumulators;
+// rows nobody writes are zero-filled.
+void assign_writers(st_layout* L) {
+  const Geom& g = L->geom;
+  std::vector<int32_t> rows;
+  for (int hc = 0; hc < (int)L->hcs.size(); ++hc) {
+    std::vector<int32_t> wk((size_t)g.T, 0), wq((size_t)g.T, 0);
+    for (const BwdItem& it : L->bwd_items) {
+      if (it.hclass != hc) continue;
+      tile_rows(it.kview, g, it.ktile, rows);
+      for (int32_t j : rows) wk[(size_t)j] += 1;
+      for (int32_t e = it.qbeg; e < it.qend; ++e) {
+        tile_rows(it.qview, g, L->q_ents[(size_t)e].qtile, rows);
+        for (int32_t i : rows) wq[(size_t)i] += 1;
+      }
+    }
+    std::vector<uint8_t> acck((size_t)g.T, 0), accq((size_t)g.T, 0);
+    for (BwdItem& it : L->bwd_items) {
+      if (it.hclass != hc) continue;
+      tile_rows(it.kview, g, it.ktile, rows);
+      bool direct = true;
+      for (int32_t j : rows) direct = direct && wk[(size_t)j] == 1;
+      it.kv_direct = direct ? 1 : 0;
+      if (!direct)
+        for (int32_t j : rows) acck[(size_t)j] = 1;
+      for (int32_t e = it.qbeg; e < it.qend; ++e) {
+        QEnt& qe = L->q_ents[(size_t)e];
+        tile_rows(it.qview, g, qe.qtile, rows);
+        bool qd = true;
+        for (int32_t i : rows) qd = qd && wq[(size_t)i] == 1;
+        qe.q_direct = qd ? 1 : 0;
+        if (!qd)
+          for (int32_t i : rows) accq[(size_t)i] = 1;
+      }
+    }
+    for (int k = 0; k < N_ROWLISTS; ++k) L->rows[hc][k].clear();
+    for (int32_t t = 0; t < g.T; ++t) {
+      if (accq[(size_t)t]) L->rows[hc][ROWS_Q_ACC].push_back(t);
+      if (acck[(size_t)t]) L->rows[hc][ROWS_K_ACC].push_back(t);
+      if (wq[(size_t)t] == 0) L->rows[hc][ROWS_Q_ZERO].push_back(t);
+      if (wk[(size_t)t] == 0) L->rows[hc][ROWS_K_ZERO].push_back(t);
+    }
+  }
+}
+
 }  // namespace
 
 st_status build_layout(const st_pattern_desc* desc, st_layout* L) {
@@ -315,7 +380,8 @@ st_status build_layout(const st_pattern_desc* desc, st_layout* L) {
         QEnt e;
         e.qtile = t.q;
         e.flag = t.flag;
-        e.pad[0] = e.pad[1] = e.pad[2] = 0;
+        e.q_direct = 0;
+        e.pad[0] = e.pad[1] = 0;
         per_k[(size_t)t.k].qs.push_back(e);
       }
       for (int32_t k = 0; k < s.nk; ++k) {
@@ -348,8 +414,11 @@ st_status build_layout(const st_pattern_desc* desc, st_layout* L) {
     p.it.qbeg = (int32_t)L->q_ents.size();
     L->q_ents.insert(L->q_ents.end(), p.qs.begin(), p.qs.end());
     p.it.qend = (int32_t)L->q_ents.size();
+    p.it.kv_direct = 0;
+    p.it.pad[0] = p.it.pad[1] = p.it.pad[2] = 0;
     L->bwd_items.push_back(p.it);
   }
+  assign_writers(L);
   return ST_OK;
 }
 

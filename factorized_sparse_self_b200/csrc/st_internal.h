@@ -61,12 +61,25 @@ struct BwdItem {
   uint8_t kview;
   uint8_t qview;
   uint8_t rule;
+  uint8_t kv_direct;   // 1: this unit alone produces dK, dV of its key tile rows
+  uint8_t pad[3];
 };
 
 struct QEnt {
   int32_t qtile;
   uint8_t flag;
-  uint8_t pad[3];
+  uint8_t q_direct;    // 1: this pair alone produces dQ of its query tile rows
+  uint8_t pad[2];
+};
+
+// Natural rows of one head class whose gradient needs a given treatment in
+// the backward prologue / epilogue (bf16 path).
+enum RowList : int {
+  ROWS_Q_ACC = 0,   // dQ accumulated in fp32 (several contributions)
+  ROWS_K_ACC = 1,   // dK, dV accumulated in fp32
+  ROWS_Q_ZERO = 2,  // dQ rows nobody writes: zero-filled
+  ROWS_K_ZERO = 3,  // dK, dV rows nobody writes: zero-filled
+  N_ROWLISTS = 4
 };
 
 // Geometry every kernel needs to map view rows to natural positions.
@@ -104,6 +117,10 @@ struct DeviceSchedule {
   int32_t n_bwd_items = 0;
   void* q_ents = nullptr;
   int32_t max_fwd_keys = 0;    // longest key list of a forward item
+  // per head class (at most 2) and row list: device array of natural rows
+  void* rows[2][N_ROWLISTS] = {{nullptr, nullptr, nullptr, nullptr},
+                               {nullptr, nullptr, nullptr, nullptr}};
+  int32_t n_rows[2][N_ROWLISTS] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
 };
 
 }  // namespace st
@@ -119,6 +136,7 @@ struct st_layout {
   std::vector<st::KeyEnt> key_ents;
   std::vector<st::BwdItem> bwd_items;
   std::vector<st::QEnt> q_ents;
+  std::vector<int32_t> rows[2][st::N_ROWLISTS];  // see st::RowList
   bool on_device = false;
   int device = -1;
   st::DeviceSchedule dev;
