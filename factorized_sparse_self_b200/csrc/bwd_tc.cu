@@ -45,7 +45,7 @@ using namespace tc;
 constexpr int NS = 2;
 constexpr int kTileBytes = kTile * 64 * 2;  // 128 x 64 bf16 = 16 KB
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsCompute = 200, kRegsIssue = 104;  // launch: 168 per thread
+constexpr uint32_t kRegsCompute = 208, kRegsIssue = 88;  // launch: 168 per thread
 static_assert(256 * kRegsCompute + 128 * kRegsIssue == kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
@@ -65,8 +65,8 @@ struct SmemBwd {
   uint8_t pt[2 * kTileBytes];    // P^T (keys x queries), two 64-query K-blocks
   uint8_t dst[2 * kTileBytes];   // dS^T, same layout
   uint8_t stage[2 * kTileBytes]; // dQ tile: fp32 in two 32-column halves, or bf16
-  float l2[NS][kTile];           // LSE_i * log2(e) of the stage's query rows
-  float dd[NS][kTile];           // D_i
+  float l2[NS][kTile];           // -LSE_i * log2(e) of the stage's query rows
+  float dd[NS][kTile];           // -D_i
   uint64_t kv_full, kv_done, full[NS], empty[NS];
   uint64_t s_full, dp_full, sdp_free, ds_ready, pds_free, dq_full, dq_free, stg_full, stg_free;
   uint64_t acc_free, out_full, kvstg_free, fin;
@@ -248,28 +248,37 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         const int cnt = x.it.qend - x.it.qbeg;
         auto issue_q = [&](int e) -> bool {
           const int s = gt % NS;
+          // schedule entries and the LSE / D rows are read before the wait for
+          // the ring stage, so that their latency stays off the critical path
+          const QEnt qe = qents[x.it.qbeg + e];
+          const int pf = (e + 2 < cnt) ? qents[x.it.qbeg + e + 2].qtile : -1;
+          float Lv[4], Dv[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int i = view_pos(g, x.it.qview, qe.qtile, lane + 32 * t);
+            const size_t at = (size_t)x.bh * g.T + (i >= 0 ? i : 0);
+            Lv[t] = __ldg(lse + at);
+            Dv[t] = __ldg(Dg + at);
+            if (i < 0) Lv[t] = Dv[t] = 0.f;
+          }
           const bool w = mbar_wait(&S.empty[s], ((gt / NS) & 1) ^ 1, wait_ns, abort);
           if (!__all_sync(0xffffffffu, w)) return false;
-          const QEnt qe = qents[x.it.qbeg + e];
           if (lane == 0) {
             mbar_arrive_expect_tx(&S.full[s], 2 * kTileBytes);
             load_tile(S.q[s], maps.q, x.it.qview, g, qe.qtile, x.bh, &S.full[s]);
             load_tile(S.dout[s], maps.dout, x.it.qview, g, qe.qtile, x.bh, &S.full[s]);
-            if (e + 2 < cnt) {  // two tiles ahead of the ring: into L2 now
-              const int pt = qents[x.it.qbeg + e + 2].qtile;
-              prefetch_tile(maps.q, x.it.qview, g, pt, x.bh);
-              prefetch_tile(maps.dout, x.it.qview, g, pt, x.bh);
+            if (pf >= 0) {  // two tiles ahead of the ring: into L2 now
+              prefetch_tile(maps.q, x.it.qview, g, pf, x.bh);
+              prefetch_tile(maps.dout, x.it.qview, g, pf, x.bh);
             }
           }
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             const int row = lane + 32 * t;
-            const int i = view_pos(g, x.it.qview, qe.qtile, row);
             // rows with an empty set (LSE = -inf) have no live pair; 0 keeps
             // their masked exponents at -inf instead of -inf + inf
-            const float L = (i >= 0) ? lse[(size_t)x.bh * g.T + i] : 0.f;
-            S.l2[s][row] = (L > -INFINITY) ? L * kLog2e : 0.f;
-            S.dd[s][row] = (i >= 0) ? Dg[(size_t)x.bh * g.T + i] : 0.f;
+            S.l2[s][row] = (Lv[t] > -INFINITY) ? -Lv[t] * kLog2e : 0.f;
+            S.dd[s][row] = -Dv[t];
           }
           mbar_arrive(&S.full[s]);
           full_last[s] = gt;
@@ -281,6 +290,14 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         const int pre = min(cnt, NS);
         int e = 0;
         for (; ok && e < pre; ++e) ok = issue_q(e);
+        // K, V of the following unit into L2 while this one runs
+        if (lane == 0 && u + (int)gridDim.x < n_units) {
+          const Unit y = unit_of(items, u + gridDim.x, NH, B, H, nclasses);
+          if (y.bh >= 0) {
+            prefetch_tile(maps.k, y.it.kview, g, y.it.ktile, y.bh);
+            prefetch_tile(maps.v, y.it.kview, g, y.it.ktile, y.bh);
+          }
+        }
         if (!ok) break;
         ok = __all_sync(0xffffffffu, mbar_wait(&S.kv_done, (n & 1) ^ 1, wait_ns, abort));
         if (!ok) break;
@@ -498,8 +515,6 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         bool w = mbar_wait(&S.s_full, gt & 1, wait_ns, abort);
         w = w && mbar_wait(&S.dp_full, gt & 1, wait_ns, abort);
         w = w && mbar_wait(&S.full[s], (gt / NS) & 1, wait_ns, abort);
-        if (gt > 0) w = w && mbar_wait(&S.pds_free, (gt - 1) & 1, wait_ns, abort);
-        if (e == 0 && n > 0) w = w && mbar_wait(&S.kvstg_free, (n - 1) & 1, wait_ns, abort);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
@@ -523,6 +538,9 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         }
         const float* l2 = S.l2[s] + wg * 64;
         const float* dd = S.dd[s] + wg * 64;
+        // P^T and dS^T of the whole row slice in registers first: the tensor
+        // core may still be reading the previous tile's from shared memory
+        uint32_t pw[8][4], dw[8][4];
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           const float4 la = *reinterpret_cast<const float4*>(l2 + ch * 8);
@@ -531,22 +549,36 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           const float4 db = *reinterpret_cast<const float4*>(dd + ch * 8 + 4);
           const float lv[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
           const float dv8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
-          uint32_t pw[4], dw[4];
 #pragma unroll
           for (int x2 = 0; x2 < 4; ++x2) {
             const int xk = ch * 8 + x2 * 2;
             float a0, a1;
-            ffma2(a0, a1, sv[xk], sv[xk + 1], scale_log2, scale_log2, -lv[2 * x2],
-                  -lv[2 * x2 + 1]);
+            ffma2(a0, a1, sv[xk], sv[xk + 1], scale_log2, scale_log2, lv[2 * x2],
+                  lv[2 * x2 + 1]);
             const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
             float t0, t1, q0, q1;
-            fadd2(t0, t1, dp[xk], dp[xk + 1], -dv8[2 * x2], -dv8[2 * x2 + 1]);
+            fadd2(t0, t1, dp[xk], dp[xk + 1], dv8[2 * x2], dv8[2 * x2 + 1]);
             fmul2(q0, q1, p0, p1, t0, t1);
-            pw[x2] = pack_bf16(p0, p1);
-            dw[x2] = pack_bf16(q0, q1);
+            pw[ch][x2] = pack_bf16(p0, p1);
+            dw[ch][x2] = pack_bf16(q0, q1);
           }
-          st_shared_v4(pt_addr + wg * kTileBytes + swz128(row, ch), pw[0], pw[1], pw[2], pw[3]);
-          st_shared_v4(ds_addr + wg * kTileBytes + swz128(row, ch), dw[0], dw[1], dw[2], dw[3]);
+        }
+        // the previous tile's dV, dK, dQ products are done with P^T, dS^T; at
+        // the start of a unit the previous unit's dK, dV staging is read too
+        w = true;
+        if (gt > 0) w = mbar_wait(&S.pds_free, (gt - 1) & 1, wait_ns, abort);
+        if (e == 0 && n > 0) w = w && mbar_wait(&S.kvstg_free, (n - 1) & 1, wait_ns, abort);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          st_shared_v4(pt_addr + wg * kTileBytes + swz128(row, ch), pw[ch][0], pw[ch][1],
+                       pw[ch][2], pw[ch][3]);
+          st_shared_v4(ds_addr + wg * kTileBytes + swz128(row, ch), dw[ch][0], dw[ch][1],
+                       dw[ch][2], dw[ch][3]);
         }
         fence_async_smem();
         tc_fence_before();

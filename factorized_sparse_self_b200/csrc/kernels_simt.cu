@@ -296,8 +296,22 @@ RowSet row_set_of(const st_layout* L) {
 }
 
 // Grid (x, B*H); d = 64 bf16 rows of 128 bytes.
-__global__ void bwd_prep_kernel(const __nv_bfloat162* __restrict__ o,
-                                const __nv_bfloat162* __restrict__ dout, float* __restrict__ Dv,
+__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
+  const uint32_t* x = reinterpret_cast<const uint32_t*>(&a);
+  const uint32_t* y = reinterpret_cast<const uint32_t*>(&b);
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 u = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x[k]));
+    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y[k]));
+    s = fmaf(u.x, v.x, s);
+    s = fmaf(u.y, v.y, s);
+  }
+  return s;
+}
+
+__global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
+                                float* __restrict__ Dv,
                                 int T, int H, int nclasses, RowSet rs, float4* __restrict__ dq_acc,
                                 float4* __restrict__ dk_acc, float4* __restrict__ dv_acc,
                                 uint4* __restrict__ dq, uint4* __restrict__ dk,
@@ -305,19 +319,37 @@ __global__ void bwd_prep_kernel(const __nv_bfloat162* __restrict__ o,
   const int bh = blockIdx.y;
   const int hc = (nclasses == 2) ? ((bh % H) & 1) : 0;
   const size_t rb = (size_t)bh * T;
-  const int lane = threadIdx.x & 31;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nwarps = (gridDim.x * blockDim.x) >> 5;
-  for (int r = warp; r < T; r += nwarps) {
-    const float2 a = __bfloat1622float2(o[(rb + r) * 32 + lane]);
-    const float2 b = __bfloat1622float2(dout[(rb + r) * 32 + lane]);
-    float sacc = fmaf(a.x, b.x, a.y * b.y);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, off);
-    if (lane == 0) Dv[rb + r] = sacc;
-  }
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int stride = gridDim.x * blockDim.x;
+  // D: eight lanes per 128-byte row (one 16-byte chunk each), four rows per
+  // warp and pass, four passes' loads in flight per thread
+  {
+    const int lane = threadIdx.x & 31, sub = lane & 7;
+    const int rstep = stride >> 3;  // rows per pass over the grid (multiple of 4)
+    const uint4* o4 = o + rb * 8;
+    const uint4* d4 = dout + rb * 8;
+    for (int rw = (tid >> 5) * 4; rw < T; rw += 4 * rstep) {  // warp-uniform
+      uint4 a[4], b[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = rw + (lane >> 3) + u * rstep;
+        a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (r < T) {
+          a[u] = __ldg(o4 + (size_t)r * 8 + sub);
+          b[u] = __ldg(d4 + (size_t)r * 8 + sub);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float sacc = dot8_bf16(a[u], b[u]);
+        sacc += __shfl_xor_sync(0xffffffffu, sacc, 4);
+        sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
+        sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
+        const int r = rw + (lane >> 3) + u * rstep;
+        if (sub == 0 && r < T) Dv[rb + r] = sacc;
+      }
+    }
+  }
   const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
   const uint4 zu = make_uint4(0u, 0u, 0u, 0u);
   {
@@ -352,17 +384,21 @@ __global__ void bwd_prep_kernel(const __nv_bfloat162* __restrict__ o,
   }
 }
 
-__device__ __forceinline__ uint2 round4(float4 a, float s) {
-  __nv_bfloat162 lo = __floats2bfloat162_rn(a.x * s, a.y * s);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(a.z * s, a.w * s);
-  return make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+__device__ __forceinline__ uint4 round8f(const float4& a, const float4& b, float s) {
+  __nv_bfloat162 w[4] = {__floats2bfloat162_rn(a.x * s, a.y * s),
+                         __floats2bfloat162_rn(a.z * s, a.w * s),
+                         __floats2bfloat162_rn(b.x * s, b.y * s),
+                         __floats2bfloat162_rn(b.z * s, b.w * s)};
+  return *reinterpret_cast<uint4*>(w);
 }
 
+// Rounds the accumulated rows: eight elements (two float4 in, 16 bytes out)
+// per thread and step.
 __global__ void bwd_finish_kernel(const float4* __restrict__ dq_acc,
                                   const float4* __restrict__ dk_acc,
                                   const float4* __restrict__ dv_acc, int T, int H, int nclasses,
-                                  RowSet rs, float scale, uint2* __restrict__ dq,
-                                  uint2* __restrict__ dk, uint2* __restrict__ dv) {
+                                  RowSet rs, float scale, uint4* __restrict__ dq,
+                                  uint4* __restrict__ dk, uint4* __restrict__ dv) {
   const int bh = blockIdx.y;
   const int hc = (nclasses == 2) ? ((bh % H) & 1) : 0;
   const size_t rb = (size_t)bh * T;
@@ -371,18 +407,18 @@ __global__ void bwd_finish_kernel(const float4* __restrict__ dq_acc,
   {
     int nr;
     const int32_t* rows = rows_of(rs, hc, ROWS_Q_ACC, nr);
-    for (int64_t x = tid; x < (int64_t)nr * 16; x += stride) {
-      const size_t e = (rb + rows[x >> 4]) * 16 + (x & 15);
-      dq[e] = round4(dq_acc[e], scale);
+    for (int64_t x = tid; x < (int64_t)nr * 8; x += stride) {
+      const size_t e = (rb + rows[x >> 3]) * 8 + (x & 7);
+      dq[e] = round8f(__ldg(dq_acc + 2 * e), __ldg(dq_acc + 2 * e + 1), scale);
     }
   }
   {
     int nr;
     const int32_t* rows = rows_of(rs, hc, ROWS_K_ACC, nr);
-    for (int64_t x = tid; x < (int64_t)nr * 16; x += stride) {
-      const size_t e = (rb + rows[x >> 4]) * 16 + (x & 15);
-      dk[e] = round4(dk_acc[e], scale);
-      dv[e] = round4(dv_acc[e], 1.f);
+    for (int64_t x = tid; x < (int64_t)nr * 8; x += stride) {
+      const size_t e = (rb + rows[x >> 3]) * 8 + (x & 7);
+      dk[e] = round8f(__ldg(dk_acc + 2 * e), __ldg(dk_acc + 2 * e + 1), scale);
+      dv[e] = round8f(__ldg(dv_acc + 2 * e), __ldg(dv_acc + 2 * e + 1), 1.f);
     }
   }
 }
@@ -498,10 +534,10 @@ cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* 
 cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* Dv, float* dq_acc,
                      float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv) {
   const int T = c.L->geom.T;
-  const int bx = std::max(1, std::min(64, (T * 32 + 255) / 256));
+  const int bx = std::max(1, std::min(64, (T + 127) / 128));
   dim3 grid(bx, c.B * c.H);
   bwd_prep_kernel<<<grid, 256, 0, c.stream>>>(
-      (const __nv_bfloat162*)o, (const __nv_bfloat162*)dout, Dv, T, c.H, c.nclasses,
+      (const uint4*)o, (const uint4*)dout, Dv, T, c.H, c.nclasses,
       row_set_of(c.L), (float4*)dq_acc, (float4*)dk_acc, (float4*)dv_acc, (uint4*)dq, (uint4*)dk,
       (uint4*)dv);
   return cudaGetLastError();
@@ -514,11 +550,11 @@ cudaError_t bwd_finish(const Call& c, const float* dq_acc, const float* dk_acc,
   for (int hc = 0; hc < (int)L->hcs.size(); ++hc)
     most = std::max(most, std::max(L->dev.n_rows[hc][ROWS_Q_ACC], L->dev.n_rows[hc][ROWS_K_ACC]));
   if (most == 0) return cudaSuccess;  // every row was written directly
-  const int bx = std::max(1, std::min(64, (most * 16 + 255) / 256));
+  const int bx = std::max(1, std::min(64, (most + 31) / 32));
   dim3 grid(bx, c.B * c.H);
   bwd_finish_kernel<<<grid, 256, 0, c.stream>>>(
       (const float4*)dq_acc, (const float4*)dk_acc, (const float4*)dv_acc, L->geom.T, c.H,
-      c.nclasses, row_set_of(L), c.scale, (uint2*)dq, (uint2*)dk, (uint2*)dv);
+      c.nclasses, row_set_of(L), c.scale, (uint4*)dq, (uint4*)dk, (uint4*)dv);
   return cudaGetLastError();
 }
 

@@ -4,8 +4,10 @@
       --B 1 --H 8 --T 16384 --l 1 --c 1 --iters 5 --warmup 2
 
 Prints one JSON line with per-call CUDA-event times of the forward attention
-launches and of the backward attention kernel, and the useful TFLOP/s
-(4 d nnz forward, 10 d nnz backward). Inputs are the seeded synthetic ones
+launches, of the backward attention kernel and of the whole forward + backward
+call pair (ms_step), and the useful TFLOP/s (4 d nnz forward, 10 d nnz
+backward). --flush writes 256 MB between iterations so that every call starts
+with a cold L2. Inputs are the seeded synthetic ones
 (bf16, std 0.5; dO ~ N(0, 1)).
 """
 from __future__ import annotations
@@ -31,6 +33,7 @@ def main():
     ap.add_argument("--iters", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--fwd-only", action="store_true")
+    ap.add_argument("--flush", action="store_true")
     a = ap.parse_args()
 
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
@@ -61,11 +64,19 @@ def main():
     for _ in range(a.warmup):
         run()
     torch.cuda.synchronize()
+    flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda") if a.flush else None
     st.st_kernel_timing(True)
-    tf, tb = [], []
+    tf, tb, ts = [], [], []
     for _ in range(a.iters):
+        if flush is not None:
+            flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
         run()
+        e1.record()
         torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
         tf.append(st.st_kernel_elapsed_ms(0))
         if not a.fwd_only:
             tb.append(st.st_kernel_elapsed_ms(1))
@@ -74,7 +85,7 @@ def main():
     if status != st.ST_OK:
         raise SystemExit(f"device status {status}")
     res = {"kind": a.kind, "mode": a.mode, "B": a.B, "H": a.H, "T": a.T, "d": a.d, "l": a.l,
-           "c": a.c, "nnz": nnz, "ms_fwd": statistics.mean(tf),
+           "c": a.c, "nnz": nnz, "ms_step": statistics.mean(ts), "ms_fwd": statistics.mean(tf),
            "fwd_tflops": 4.0 * a.d * nnz / (statistics.mean(tf) * 1e-3) / 1e12}
     if tb:
         res["ms_bwd_kernel"] = statistics.mean(tb)
