@@ -7,26 +7,29 @@
 //   dP^T = V dO^T
 //   P^T  = exp(scale S^T - LSE_i) on the live pairs, 0 elsewhere
 //   dS^T = P^T (dP^T - D_i),      D_i = dO_i . O_i (prologue kernel)
-//   dV  += P^T dO                 (M=128, N=64, K=128)
-//   dK  += dS^T Q
+//   dV  += P^T dO                 (M=128, N=64, K=128; P^T read from TMEM)
+//   dK  += dS^T Q                 (dS^T from shared memory)
 //   dQ_i = dS K
 // dV and dK stay in TMEM for a whole work unit (a key tile, or a chunk of a
 // long key column). A gradient tile whose rows no other unit (for dK, dV) or
 // pair (for dQ) touches is scaled, rounded to bf16 and TMA-stored straight
 // into the output; every other tile is TMA reduce-added into an fp32
-// accumulator, which a later kernel scales and rounds.
+// accumulator, which a later kernel scales and rounds. K and V are
+// double-buffered across units.
 //
-// Persistent CTAs, one per SM, each walking a strided share of the work units
-// (longest first). Warpgroup roles:
+// Persistent CTAs, one per SM. The producer warp claims work units (sorted
+// longest first) from a global counter and publishes them to the other roles
+// through a small shared-memory ring, so that every CTA takes the next unit
+// when it is ready for one. Warpgroup roles:
 //   warpgroups 0, 1  compute: thread = key row = TMEM lane for S^T / dP^T;
 //                    warpgroup w owns query columns 64w .. 64w+63 of every
-//                    tile, the dQ columns 32w .. 32w+31, and drains dK (w = 0)
-//                    or dV (w = 1) at the end of a unit;
-//   warpgroup 2      warp 8 TMA producer (K, V per unit; Q, dO per query
-//                    tile into a 2-stage ring, with LSE and D by plain loads),
-//                    warp 9 TMEM owner and MMA issuer, warp 10 reducer (TMA
-//                    reduce-adds of the staged dQ, dK, dV tiles, so that no
-//                    compute warp waits on a bulk copy).
+//                    tile, the dQ columns 32w .. 32w+31, and writes out dK
+//                    (w = 0) or dV (w = 1) at the end of a unit;
+//   warpgroup 2      warp 8 TMA producer (K, V per unit into two buffers; Q,
+//                    dO per query tile into a 2-stage ring, with LSE and D by
+//                    plain loads), warp 9 TMEM owner and MMA issuer, warp 10
+//                    writer (TMA reduce-adds or stores of the staged dQ, dK,
+//                    dV tiles, so that no compute warp waits on a bulk copy).
 // The MMA warp issues S, dP of the next tile as soon as the compute warps hold
 // the current tile's in registers, ahead of dV, dK, dQ of the current tile,
 // so the exponentials overlap the tensor pipe. All waits are bounded.
@@ -43,12 +46,14 @@ namespace {
 using namespace tc;
 
 constexpr int NS = 2;
+constexpr int kSched = 4;                   // published work units in flight
 constexpr int kTileBytes = kTile * 64 * 2;  // 128 x 64 bf16 = 16 KB
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsCompute = 208, kRegsIssue = 88;  // launch: 168 per thread
+constexpr uint32_t kRegsCompute = 200, kRegsIssue = 104;  // launch: 168 per thread
 static_assert(256 * kRegsCompute + 128 * kRegsIssue == kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
+constexpr uint32_t kColPT = 448;  // P^T as packed bf16 pairs, 64 columns
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdMaps {
@@ -58,18 +63,20 @@ struct BwdMaps {
 };
 
 struct SmemBwd {
-  uint8_t k[kTileBytes];
-  uint8_t v[kTileBytes];
+  uint8_t k[2][kTileBytes];
+  uint8_t v[2][kTileBytes];
   uint8_t q[NS][kTileBytes];
   uint8_t dout[NS][kTileBytes];
-  uint8_t pt[2 * kTileBytes];    // P^T (keys x queries), two 64-query K-blocks
-  uint8_t dst[2 * kTileBytes];   // dS^T, same layout
+  uint8_t dst[2 * kTileBytes];   // dS^T (keys x queries), two 64-query K-blocks
   uint8_t stage[2 * kTileBytes]; // dQ tile: fp32 in two 32-column halves, or bf16
+  uint8_t kvst[2 * kTileBytes];  // dK tile at the end of a unit (dV goes through dst)
   float l2[NS][kTile];           // -LSE_i * log2(e) of the stage's query rows
   float dd[NS][kTile];           // -D_i
-  uint64_t kv_full, kv_done, full[NS], empty[NS];
+  uint64_t kv_full[2], kv_done[2], full[NS], empty[NS];
   uint64_t s_full, dp_full, sdp_free, ds_ready, pds_free, dq_full, dq_free, stg_full, stg_free;
-  uint64_t acc_free, out_full, kvstg_free, fin;
+  uint64_t acc_full, acc_free, out_full, kvstg_free, fin;
+  uint64_t sched_full[kSched], sched_empty[kSched];
+  int sched[kSched];             // work unit of each slot (n_units: no more work)
   uint32_t tmem_base;
   int abort;
 };
@@ -191,17 +198,26 @@ __device__ __forceinline__ Unit unit_of(const BwdItem* items, int u, int NH, int
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __restrict__ items,
               int n_units, int NH, const QEnt* __restrict__ qents, int B, int H, int nclasses,
-              float scale, float scale_log2, const float* __restrict__ lse, const float* __restrict__ Dg,
-              int* status, uint64_t wait_ns) {
-  extern __shared__ uint8_t smem_raw[];
-  SmemBwd& S = *reinterpret_cast<SmemBwd*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~uintptr_t(1023));
+              float scale, float scale_log2, const float* __restrict__ lse,
+              const float* __restrict__ Dg, int* sched_counter, int* status,
+              uint64_t wait_ns) {
+  // The shared-memory plan fills the 227 KB a CTA may hold, with no room to
+  // realign: the swizzled tiles need the dynamic window at a 1024-byte
+  // boundary (where it starts when the kernel has no static shared memory).
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) set_status(status, ST_ERR_UNSUPPORTED);
+    return;
+  }
+  SmemBwd& S = *reinterpret_cast<SmemBwd*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &S.abort;
 
   if (threadIdx.x == 0) {
-    mbar_init(&S.kv_full, 1);
-    mbar_init(&S.kv_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.kv_full[b], 1);
+      mbar_init(&S.kv_done[b], 1);
+    }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&S.full[s], 33);  // expect_tx arrive + 32 producer lanes
       mbar_init(&S.empty[s], 1);
@@ -215,10 +231,15 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     mbar_init(&S.dq_free, 256);
     mbar_init(&S.stg_full, 256);
     mbar_init(&S.stg_free, 1);
+    mbar_init(&S.acc_full, 1);
     mbar_init(&S.acc_free, 256);
     mbar_init(&S.out_full, 256);
     mbar_init(&S.kvstg_free, 1);
     mbar_init(&S.fin, 1);
+    for (int k = 0; k < kSched; ++k) {
+      mbar_init(&S.sched_full[k], 1);
+      mbar_init(&S.sched_empty[k], 10);  // MMA lane, reducer lane, 8 compute warps
+    }
     S.abort = 0;
     fence_mbar_init();
   }
@@ -233,6 +254,18 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     *abort = 1;
     set_status(status, ST_ERR_DEVICE_TIMEOUT);
   };
+  // Next published unit for a consuming role; `arrive` releases the slot
+  // (one arrival per consuming warp).
+  int sk = 0;
+  auto next_unit = [&](int& u, bool arrive) -> bool {
+    const int k = sk % kSched;
+    const bool w = mbar_wait(&S.sched_full[k], (sk / kSched) & 1, wait_ns, abort);
+    if (!w) return false;
+    u = *reinterpret_cast<volatile int*>(&S.sched[k]);
+    if (arrive) mbar_arrive(&S.sched_empty[k]);
+    ++sk;
+    return true;
+  };
 
   if (warp >= 8) {
     regs_decrease<kRegsIssue>();
@@ -241,10 +274,34 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       int full_last[NS] = {-1, -1};
       int kv_last = -1;
       bool ok = true;
-      int gt = 0, n = 0;
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-        const Unit x = unit_of(items, u, NH, B, H, nclasses);
-        if (x.bh < 0) continue;
+      int gt = 0, n = 0, pub = 0;
+      // claims units until one has a head of its class (bh >= 0)
+      auto claim = [&]() -> int {
+        int u = 0;
+        for (;;) {
+          if (lane == 0) u = atomicAdd(sched_counter, 1);
+          u = __shfl_sync(0xffffffffu, u, 0);
+          if (u >= n_units) return n_units;
+          if (unit_of(items, u, NH, B, H, nclasses).bh >= 0) return u;
+        }
+      };
+      auto publish = [&](int u) -> bool {
+        const int k = pub % kSched;
+        const bool w = mbar_wait(&S.sched_empty[k], ((pub / kSched) & 1) ^ 1, wait_ns, abort);
+        if (!__all_sync(0xffffffffu, w)) return false;
+        if (lane == 0) {
+          S.sched[k] = u;
+          mbar_arrive(&S.sched_full[k]);
+        }
+        ++pub;
+        return true;
+      };
+      int cur = claim();
+      while (ok && cur < n_units) {
+        ok = publish(cur);
+        if (!ok) break;
+        const int nxt = claim();
+        const Unit x = unit_of(items, cur, NH, B, H, nclasses);
         const int cnt = x.it.qend - x.it.qbeg;
         auto issue_q = [&](int e) -> bool {
           const int s = gt % NS;
@@ -285,34 +342,33 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           ++gt;
           return true;
         };
-        // the first query tiles of the unit may load while the previous unit
-        // still holds the K / V buffers
-        const int pre = min(cnt, NS);
-        int e = 0;
-        for (; ok && e < pre; ++e) ok = issue_q(e);
-        // K, V of the following unit into L2 while this one runs
-        if (lane == 0 && u + (int)gridDim.x < n_units) {
-          const Unit y = unit_of(items, u + gridDim.x, NH, B, H, nclasses);
-          if (y.bh >= 0) {
+        // K, V first: buffer n & 1 was last read by this CTA's unit n - 2,
+        // normally finished by the time the producer gets here
+        const int kb = n & 1;
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&S.kv_done[kb], ((n >> 1) & 1) ^ 1, wait_ns, abort));
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&S.kv_full[kb], 2 * kTileBytes);
+          load_tile(S.k[kb], maps.k, x.it.kview, g, x.it.ktile, x.bh, &S.kv_full[kb]);
+          load_tile(S.v[kb], maps.v, x.it.kview, g, x.it.ktile, x.bh, &S.kv_full[kb]);
+          if (nxt < n_units) {  // K, V of the following unit into L2 meanwhile
+            const Unit y = unit_of(items, nxt, NH, B, H, nclasses);
             prefetch_tile(maps.k, y.it.kview, g, y.it.ktile, y.bh);
             prefetch_tile(maps.v, y.it.kview, g, y.it.ktile, y.bh);
           }
         }
-        if (!ok) break;
-        ok = __all_sync(0xffffffffu, mbar_wait(&S.kv_done, (n & 1) ^ 1, wait_ns, abort));
-        if (!ok) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&S.kv_full, 2 * kTileBytes);
-          load_tile(S.k, maps.k, x.it.kview, g, x.it.ktile, x.bh, &S.kv_full);
-          load_tile(S.v, maps.v, x.it.kview, g, x.it.ktile, x.bh, &S.kv_full);
-        }
         kv_last = n;
-        for (; ok && e < cnt; ++e) ok = issue_q(e);
+        for (int e = 0; ok && e < cnt; ++e) ok = issue_q(e);
         ++n;
+        cur = nxt;
       }
+      if (ok) ok = publish(n_units);  // no more work
       if (!ok && lane == 0) fail();
       if (lane == 0) {
-        if (kv_last >= 0 && !mbar_wait(&S.kv_full, kv_last & 1, wait_ns, abort)) fail();
+        // the last K / V loads of both buffers have landed before the exit
+        for (int m = max(kv_last - 1, 0); m <= kv_last; ++m)
+          if (!mbar_wait(&S.kv_full[m & 1], (m >> 1) & 1, wait_ns, abort)) fail();
         for (int s = 0; s < NS; ++s)
           if (full_last[s] >= 0 &&
               !mbar_wait(&S.full[s], (full_last[s] / NS) & 1, wait_ns, abort))
@@ -324,8 +380,8 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         const uint32_t idSS = idesc_bf16(128, 128, false, false);
         const uint32_t idKM = idesc_bf16(128, 64, false, true);  // A K-major, B MN-major
         const uint32_t idMM = idesc_bf16(128, 64, true, true);   // A MN-major, B MN-major
-        const uint32_t k_addr = smem_u32(S.k), v_addr = smem_u32(S.v);
-        const uint32_t pt_addr = smem_u32(S.pt), ds_addr = smem_u32(S.dst);
+        const uint32_t ds_addr = smem_u32(S.dst);
+        uint32_t k_addr = 0, v_addr = 0;
         bool ok = true;
         int gt = 0, n = 0;
         auto issue_s_dp = [&](int t) -> bool {
@@ -345,11 +401,19 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           mma_commit(&S.dp_full);
           return true;
         };
-        for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        for (;;) {
+          int u = 0;
+          if (!next_unit(u, true)) {
+            ok = false;
+            break;
+          }
+          if (u >= n_units) break;
           const Unit x = unit_of(items, u, NH, B, H, nclasses);
-          if (x.bh < 0) continue;
           const int cnt = x.it.qend - x.it.qbeg;
-          ok = mbar_wait(&S.kv_full, n & 1, wait_ns, abort);
+          const int kb = n & 1;
+          k_addr = smem_u32(S.k[kb]);
+          v_addr = smem_u32(S.v[kb]);
+          ok = mbar_wait(&S.kv_full[kb], (n >> 1) & 1, wait_ns, abort);
           if (ok) ok = issue_s_dp(gt);
           for (int e = 0; ok && e < cnt; ++e, ++gt) {
             const int s = gt % NS;
@@ -372,17 +436,17 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             }
             tc_fence_after();
             const uint32_t q_addr = smem_u32(S.q[s]), o_addr = smem_u32(S.dout[s]);
-            // dV += P^T dO ; dK += dS^T Q   (K = 128 queries, 8 steps of 16)
+            // dV += P^T dO (P^T from TMEM), dK += dS^T Q: K = 128 queries in 8
+            // steps of 16, the two accumulation chains interleaved
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tmem + kColDV,
-                     sdesc(pt_addr + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
-                     sdesc(o_addr + kk * 2048, 16384, 1024), idKM, (e > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t acc = (e > 0 || kk > 0) ? 1u : 0u;
+              mma_ts(tmem + kColDV, tmem + kColPT + kk * 8, sdesc(o_addr + kk * 2048, 16384, 1024),
+                     idKM, acc);
               mma_ss(tmem + kColDK,
                      sdesc(ds_addr + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
-                     sdesc(q_addr + kk * 2048, 16384, 1024), idKM, (e > 0 || kk > 0) ? 1u : 0u);
+                     sdesc(q_addr + kk * 2048, 16384, 1024), idKM, acc);
+            }
             mma_commit(&S.empty[s]);  // Q, dO of this stage are no longer read
             if (gt > 0 && !mbar_wait(&S.dq_free, (gt - 1) & 1, wait_ns, abort)) {
               ok = false;
@@ -398,7 +462,8 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             mma_commit(&S.pds_free);
           }
           if (!ok) break;
-          mma_commit(&S.kv_done);
+          mma_commit(&S.kv_done[n & 1]);
+          mma_commit(&S.acc_full);
           ++n;
         }
         if (!ok) fail();
@@ -422,9 +487,14 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           mbar_arrive(&S.stg_free);
           return true;
         };
-        for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        for (;;) {
+          int u = 0;
+          if (!next_unit(u, true)) {
+            ok = false;
+            break;
+          }
+          if (u >= n_units) break;
           const Unit x = unit_of(items, u, NH, B, H, nclasses);
-          if (x.bh < 0) continue;
           const int cnt = x.it.qend - x.it.qbeg;
           for (int e = 0; ok && e < cnt; ++e, ++gt) {
             if (gt > 0 && !reduce_dq(gt - 1)) {
@@ -443,10 +513,10 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             break;
           }
           if (x.it.kv_direct) {
-            store_tile(maps.dko, x.it.kview, g, x.it.ktile, x.bh, S.pt);
+            store_tile(maps.dko, x.it.kview, g, x.it.ktile, x.bh, S.kvst);
             store_tile(maps.dvo, x.it.kview, g, x.it.ktile, x.bh, S.dst);
           } else {
-            reduce_tile(maps.dk, x.it.kview, g, x.it.ktile, x.bh, S.pt);
+            reduce_tile(maps.dk, x.it.kview, g, x.it.ktile, x.bh, S.kvst);
             reduce_tile(maps.dv, x.it.kview, g, x.it.ktile, x.bh, S.dst);
           }
           bulk_commit();
@@ -467,7 +537,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     const int row = lg * 32 + lane;              // key row (S^T, dP^T) / query row (dQ)
     const uint32_t tl = (uint32_t)(lg * 32) << 16;
     bool ok = true;
-    const uint32_t pt_addr = smem_u32(S.pt), ds_addr = smem_u32(S.dst);
+    const uint32_t ds_addr = smem_u32(S.dst);
     const uint32_t st_addr = smem_u32(S.stage);
     int gt = 0, n = 0;
     int pend_direct = 0;  // q_direct of the tile whose dQ is pending
@@ -503,9 +573,17 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       return true;
     };
 
-    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+    for (;;) {
+      int u = 0;
+      const bool got = next_unit(u, false);
+      __syncwarp();
+      if (lane == 0 && got) mbar_arrive(&S.sched_empty[(sk - 1) % kSched]);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      if (u >= n_units) break;
       const Unit x = unit_of(items, u, NH, B, H, nclasses);
-      if (x.bh < 0) continue;
       const BwdItem& it = x.it;
       const int cnt = it.qend - it.qbeg;
       const int j = view_pos(g, it.kview, it.ktile, row);
@@ -564,7 +642,8 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           }
         }
         // the previous tile's dV, dK, dQ products are done with P^T, dS^T; at
-        // the start of a unit the previous unit's dK, dV staging is read too
+        // the start of a unit the writer has also read the previous unit's
+        // dK, dV staging (dV sits in the dS^T buffer)
         w = true;
         if (gt > 0) w = mbar_wait(&S.pds_free, (gt - 1) & 1, wait_ns, abort);
         if (e == 0 && n > 0) w = w && mbar_wait(&S.kvstg_free, (n - 1) & 1, wait_ns, abort);
@@ -573,13 +652,12 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           break;
         }
         tc_fence_after();
+        tmem_st32(tmem + tl + kColPT + wg * 32, &pw[0][0]);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          st_shared_v4(pt_addr + wg * kTileBytes + swz128(row, ch), pw[ch][0], pw[ch][1],
-                       pw[ch][2], pw[ch][3]);
+        for (int ch = 0; ch < 8; ++ch)
           st_shared_v4(ds_addr + wg * kTileBytes + swz128(row, ch), dw[ch][0], dw[ch][1],
                        dw[ch][2], dw[ch][3]);
-        }
+        tmem_wait_st();
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(&S.ds_ready);
@@ -590,8 +668,8 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         pend_direct = qe.q_direct;
       }
       if (!ok) break;
-      // ---- end of unit: dK (warpgroup 0) or dV (warpgroup 1) -> reduce-add ----
-      bool w = mbar_wait(&S.kv_done, n & 1, wait_ns, abort);
+      // ---- end of unit: dK (warpgroup 0) or dV (warpgroup 1) out of TMEM ----
+      bool w = mbar_wait(&S.acc_full, n & 1, wait_ns, abort);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
@@ -603,7 +681,9 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&S.acc_free);
-      const uint32_t dst = wg ? ds_addr : pt_addr;
+      // stage for the writer warp: dK in its own buffer, dV in the dS^T buffer
+      // (free: every product of the unit has completed)
+      const uint32_t dst = wg ? ds_addr : smem_u32(S.kvst);
       if (it.kv_direct) {
         const float sc = wg ? 1.f : scale;  // dK carries the softmax scale, dV none
 #pragma unroll
@@ -637,7 +717,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
 
 cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, const float* lse,
                    const void* dout, const float* D, float* dq_acc, float* dk_acc,
-                   float* dv_acc, void* dq, void* dk, void* dv) {
+                   float* dv_acc, void* dq, void* dk, void* dv, int* sched_counter) {
   const st_layout* L = c.L;
   const int BH = c.B * c.H;
   if (L->dev.n_bwd_items == 0) return cudaSuccess;
@@ -653,7 +733,8 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, c
       !make_view_maps(maps.dko, dk, false, L->geom, BH, c.d) ||
       !make_view_maps(maps.dvo, dv, false, L->geom, BH, c.d))
     return cudaErrorInvalidValue;
-  const size_t smem = sizeof(SmemBwd) + 1024;
+  const size_t smem = sizeof(SmemBwd);
+  static_assert(sizeof(SmemBwd) <= 227 * 1024, "shared memory plan exceeds a CTA's 227 KB");
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -673,7 +754,7 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, c
   bwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
       maps, L->geom, (const BwdItem*)L->dev.bwd_items, (int)units, NH,
       (const QEnt*)L->dev.q_ents, c.B, c.H, c.nclasses, c.scale, c.scale * kLog2e, lse, D,
-      c.status,
+      sched_counter, c.status,
       c.wait_ns);
   err = cudaGetLastError();
   record_end(c);

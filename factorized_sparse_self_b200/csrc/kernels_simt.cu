@@ -315,8 +315,9 @@ __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __rest
                                 int T, int H, int nclasses, RowSet rs, float4* __restrict__ dq_acc,
                                 float4* __restrict__ dk_acc, float4* __restrict__ dv_acc,
                                 uint4* __restrict__ dq, uint4* __restrict__ dk,
-                                uint4* __restrict__ dv) {
+                                uint4* __restrict__ dv, int* __restrict__ sched_counter) {
   const int bh = blockIdx.y;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *sched_counter = 0;
   const int hc = (nclasses == 2) ? ((bh % H) & 1) : 0;
   const size_t rb = (size_t)bh * T;
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
@@ -532,14 +533,15 @@ cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* 
 }
 
 cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* Dv, float* dq_acc,
-                     float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv) {
+                     float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv,
+                     int* sched_counter) {
   const int T = c.L->geom.T;
   const int bx = std::max(1, std::min(64, (T + 127) / 128));
   dim3 grid(bx, c.B * c.H);
   bwd_prep_kernel<<<grid, 256, 0, c.stream>>>(
       (const uint4*)o, (const uint4*)dout, Dv, T, c.H, c.nclasses,
       row_set_of(c.L), (float4*)dq_acc, (float4*)dk_acc, (float4*)dv_acc, (uint4*)dq, (uint4*)dk,
-      (uint4*)dv);
+      (uint4*)dv, sched_counter);
   return cudaGetLastError();
 }
 

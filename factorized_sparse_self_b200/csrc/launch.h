@@ -47,8 +47,11 @@ cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* 
 // zero-fills the output rows nobody writes; bwd_finish rounds the accumulated
 // rows into dq, dk, dv (scale applied to dQ and dK). Rows that a single
 // backward unit produces are written by the tensor-core kernel itself.
+// bwd_prep also zeroes the work counter the tensor-core kernel claims its
+// units from.
 cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* D, float* dq_acc,
-                     float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv);
+                     float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv,
+                     int* sched_counter);
 cudaError_t bwd_finish(const Call& c, const float* dq_acc, const float* dk_acc,
                        const float* dv_acc, void* dq, void* dk, void* dv);
 
@@ -57,7 +60,8 @@ cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, v
                    float* lse, int force_timeout);
 cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v,
                    const float* lse, const void* dout, const float* D, float* dq_acc,
-                   float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv);
+                   float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv,
+                   int* sched_counter);
 
 }  // namespace st
 

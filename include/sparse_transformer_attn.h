@@ -144,7 +144,7 @@ st_status st_sparse_attn_bwd_workspace(const st_layout* layout, st_dtype dtype, 
  * V, the forward's O and LSE, and the upstream gradient dout. P is recomputed
  * as exp(s - LSE) on live tiles; D_i = dout_i . O_i. The workspace (device
  * memory, at least st_sparse_attn_bwd_workspace bytes, 256-byte aligned) is
- * overwritten; it holds the fp32 accumulators and D. Returns
+ * overwritten; it holds D, the fp32 accumulators and a work counter. Returns
  * ST_ERR_WORKSPACE if it is missing or too small. */
 st_status st_sparse_attn_bwd(const st_layout* layout, st_dtype dtype, int32_t B, int32_t H,
                              int32_t T, int32_t d, float scale, const void* q, const void* k,
@@ -162,7 +162,7 @@ st_status st_sparse_attn_bwd(const st_layout* layout, st_dtype dtype, int32_t B,
  * memory that every GPU which loads the library holds until the process
  * exits. It never allocates.
  *  - Limit: st_sparse_attn_bwd_workspace bytes for these sizes must not
- *    exceed 64 MiB (bf16: B*H*T*(4 + 12*d) bytes, rounded up); larger
+ *    exceed 64 MiB (bf16: B*H*T*(4 + 12*d) + 256 bytes, rounded up); larger
  *    calls return ST_ERR_WORKSPACE before any launch.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
