@@ -300,7 +300,10 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       while (ok && cur < n_units) {
         ok = publish(cur);
         if (!ok) break;
-        const int nxt = claim();
+        // the claim of the following unit goes out now; its answer is first
+        // needed once this unit's K, V and first query tile are on their way
+        int ticket = 0;
+        if (lane == 0) ticket = atomicAdd(sched_counter, 1);
         const Unit x = unit_of(items, cur, NH, B, H, nclasses);
         const int cnt = x.it.qend - x.it.qbeg;
         auto issue_q = [&](int e) -> bool {
@@ -342,24 +345,34 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           ++gt;
           return true;
         };
-        // K, V first: buffer n & 1 was last read by this CTA's unit n - 2,
-        // normally finished by the time the producer gets here
-        const int kb = n & 1;
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(&S.kv_done[kb], ((n >> 1) & 1) ^ 1, wait_ns, abort));
-        if (!ok) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&S.kv_full[kb], 2 * kTileBytes);
-          load_tile(S.k[kb], maps.k, x.it.kview, g, x.it.ktile, x.bh, &S.kv_full[kb]);
-          load_tile(S.v[kb], maps.v, x.it.kview, g, x.it.ktile, x.bh, &S.kv_full[kb]);
-          if (nxt < n_units) {  // K, V of the following unit into L2 meanwhile
-            const Unit y = unit_of(items, nxt, NH, B, H, nclasses);
-            prefetch_tile(maps.k, y.it.kview, g, y.it.ktile, y.bh);
-            prefetch_tile(maps.v, y.it.kview, g, y.it.ktile, y.bh);
+        // K, V of a unit go into buffer n & 1 (n counts this CTA's units),
+        // last read by unit n - 2. They are normally loaded one unit ahead,
+        // below; only the CTA's first unit loads its own here.
+        auto load_kv = [&](int m, const Unit& y) -> bool {
+          const int kb = m & 1;
+          const bool w = mbar_wait(&S.kv_done[kb], ((m >> 1) & 1) ^ 1, wait_ns, abort);
+          if (!__all_sync(0xffffffffu, w)) return false;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&S.kv_full[kb], 2 * kTileBytes);
+            load_tile(S.k[kb], maps.k, y.it.kview, g, y.it.ktile, y.bh, &S.kv_full[kb]);
+            load_tile(S.v[kb], maps.v, y.it.kview, g, y.it.ktile, y.bh, &S.kv_full[kb]);
           }
-        }
-        kv_last = n;
-        for (int e = 0; ok && e < cnt; ++e) ok = issue_q(e);
+          kv_last = m;
+          return true;
+        };
+        if (kv_last < n) ok = load_kv(n, x);
+        if (!ok) break;
+        if (cnt > 0) ok = issue_q(0);
+        int nxt = __shfl_sync(0xffffffffu, ticket, 0);
+        if (nxt >= n_units)
+          nxt = n_units;
+        else if (unit_of(items, nxt, NH, B, H, nclasses).bh < 0)
+          nxt = claim();
+        if (ok && cnt > 1) ok = issue_q(1);
+        // the following unit's K, V as soon as unit n - 1 has released their
+        // buffer: by now its last tiles have passed through the ring
+        if (ok && nxt < n_units) ok = load_kv(n + 1, unit_of(items, nxt, NH, B, H, nclasses));
+        for (int e = 2; ok && e < cnt; ++e) ok = issue_q(e);
         ++n;
         cur = nxt;
       }
@@ -747,12 +760,18 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, c
   }
   const int sms = sm_count();
   const int NH = heads_per_class(c);
-  const long long units = (long long)L->dev.n_bwd_items * NH;
+  // Cut accumulating items finer while the longest unit would exceed half of
+  // a CTA's share of all tile pairs (few units per CTA: the tail would be one
+  // long unit).
+  const double share = (double)L->dev.q_ents_total * NH / sms;
+  int f = 0;
+  while (f < 2 && L->dev.max_split_len[f] > 0.5 * share) ++f;
+  const long long units = (long long)L->dev.n_bwd_split[f] * NH;
   if (units > 0x7fffffff) return cudaErrorInvalidValue;
   const int grid = (int)std::min<long long>(units, sms);
   record_begin(c);
   bwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
-      maps, L->geom, (const BwdItem*)L->dev.bwd_items, (int)units, NH,
+      maps, L->geom, (const BwdItem*)L->dev.bwd_split[f], (int)units, NH,
       (const QEnt*)L->dev.q_ents, c.B, c.H, c.nclasses, c.scale, c.scale * kLog2e, lse, D,
       sched_counter, c.status,
       c.wait_ns);

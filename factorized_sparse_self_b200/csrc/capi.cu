@@ -60,6 +60,7 @@ void free_device(st_layout* L) {
   for (int p = 0; p < 2; ++p) cudaFree(L->dev.fwd_items[p]);
   cudaFree(L->dev.key_ents);
   cudaFree(L->dev.bwd_items);
+  for (int f = 1; f < 3; ++f) cudaFree(L->dev.bwd_split[f]);
   cudaFree(L->dev.q_ents);
   for (int hc = 0; hc < 2; ++hc)
     for (int k = 0; k < N_ROWLISTS; ++k) cudaFree(L->dev.rows[hc][k]);
@@ -173,6 +174,17 @@ st_status st_pattern_layout(const st_pattern_desc* desc, st_layout** out, void* 
   if (e == cudaSuccess) e = upload(&L->dev.bwd_items, L->bwd_items, cs);
   if (e == cudaSuccess) e = upload(&L->dev.q_ents, L->q_ents, cs);
   L->dev.n_bwd_items = (int32_t)L->bwd_items.size();
+  L->dev.bwd_split[0] = L->dev.bwd_items;
+  L->dev.n_bwd_split[0] = L->dev.n_bwd_items;
+  for (int f = 1; f < 3 && e == cudaSuccess; ++f) {
+    e = upload(&L->dev.bwd_split[f], L->bwd_split[f - 1], cs);
+    L->dev.n_bwd_split[f] = (int32_t)L->bwd_split[f - 1].size();
+  }
+  for (int f = 0; f < 3; ++f) {
+    const std::vector<BwdItem>& v = f == 0 ? L->bwd_items : L->bwd_split[f - 1];
+    L->dev.max_split_len[f] = v.empty() ? 0 : v.front().qend - v.front().qbeg;
+  }
+  L->dev.q_ents_total = (int64_t)L->q_ents.size();
   for (int hc = 0; hc < (int)L->hcs.size() && e == cudaSuccess; ++hc)
     for (int k = 0; k < N_ROWLISTS && e == cudaSuccess; ++k) {
       e = upload(&L->dev.rows[hc][k], L->rows[hc][k], cs);

@@ -419,6 +419,27 @@ st_status build_layout(const st_pattern_desc* desc, st_layout* L) {
     L->bwd_items.push_back(p.it);
   }
   assign_writers(L);
+  // Finer cuts of the accumulating items, for launches with few units per
+  // CTA: a key tile that already has several writers may take more (each part
+  // reduce-adds its dK, dV partial); direct items stay whole.
+  for (int f = 0; f < 2; ++f) {
+    const int32_t parts = f == 0 ? 2 : 4;
+    std::vector<BwdItem>& out = L->bwd_split[f];
+    out.clear();
+    for (const BwdItem& it : L->bwd_items) {
+      const int32_t nq = it.qend - it.qbeg;
+      const int32_t np = (it.kv_direct || nq < 2) ? 1 : std::min(parts, nq);
+      for (int32_t x = 0; x < np; ++x) {
+        BwdItem part = it;
+        part.qbeg = it.qbeg + (int32_t)((int64_t)nq * x / np);
+        part.qend = it.qbeg + (int32_t)((int64_t)nq * (x + 1) / np);
+        out.push_back(part);
+      }
+    }
+    std::stable_sort(out.begin(), out.end(), [](const BwdItem& a, const BwdItem& b) {
+      return a.qend - a.qbeg > b.qend - b.qbeg;
+    });
+  }
   return ST_OK;
 }
 

@@ -115,6 +115,12 @@ struct DeviceSchedule {
   void* key_ents = nullptr;
   void* bwd_items = nullptr;
   int32_t n_bwd_items = 0;
+  // the backward items with every accumulating (not direct) item of two or
+  // more query tiles further cut into 2 and into 4 parts; index 0 is bwd_items
+  void* bwd_split[3] = {nullptr, nullptr, nullptr};
+  int32_t n_bwd_split[3] = {0, 0, 0};
+  int32_t max_split_len[3] = {0, 0, 0};  // most query tiles of one item
+  int64_t q_ents_total = 0;
   void* q_ents = nullptr;
   int32_t max_fwd_keys = 0;    // longest key list of a forward item
   // per head class (at most 2) and row list: device array of natural rows
@@ -135,6 +141,7 @@ struct st_layout {
   std::vector<st::FwdItem> fwd_items[2];
   std::vector<st::KeyEnt> key_ents;
   std::vector<st::BwdItem> bwd_items;
+  std::vector<st::BwdItem> bwd_split[2];  // parts of 2 and of 4 (see DeviceSchedule)
   std::vector<st::QEnt> q_ents;
   std::vector<int32_t> rows[2][st::N_ROWLISTS];  // see st::RowList
   bool on_device = false;

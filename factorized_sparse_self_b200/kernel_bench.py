@@ -70,6 +70,7 @@ def main():
     for _ in range(a.iters):
         if flush is not None:
             flush.zero_()
+        torch.cuda._sleep(400000)  # the host queues the calls before the GPU reaches them
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
