@@ -275,14 +275,16 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       int kv_last = -1;
       bool ok = true;
       int gt = 0, n = 0, pub = 0;
-      // claims units until one has a head of its class (bh >= 0)
-      auto claim = [&]() -> int {
-        int u = 0;
+      // The CTA's first unit is blockIdx.x (the longest units spread one per
+      // CTA); later ones come from the counter, offset by the grid. Units
+      // without a head of their class are skipped.
+      auto valid = [&](int u) -> int {
         for (;;) {
-          if (lane == 0) u = atomicAdd(sched_counter, 1);
-          u = __shfl_sync(0xffffffffu, u, 0);
           if (u >= n_units) return n_units;
           if (unit_of(items, u, NH, B, H, nclasses).bh >= 0) return u;
+          int t = 0;
+          if (lane == 0) t = atomicAdd(sched_counter, 1);
+          u = (int)gridDim.x + __shfl_sync(0xffffffffu, t, 0);
         }
       };
       auto publish = [&](int u) -> bool {
@@ -296,12 +298,12 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         ++pub;
         return true;
       };
-      int cur = claim();
+      int cur = valid(blockIdx.x);
       while (ok && cur < n_units) {
         ok = publish(cur);
         if (!ok) break;
         // the claim of the following unit goes out now; its answer is first
-        // needed once this unit's K, V and first query tile are on their way
+        // needed once this unit's K, V are on their way
         int ticket = 0;
         if (lane == 0) ticket = atomicAdd(sched_counter, 1);
         const Unit x = unit_of(items, cur, NH, B, H, nclasses);
@@ -363,11 +365,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         if (kv_last < n) ok = load_kv(n, x);
         if (!ok) break;
         if (cnt > 0) ok = issue_q(0);
-        int nxt = __shfl_sync(0xffffffffu, ticket, 0);
-        if (nxt >= n_units)
-          nxt = n_units;
-        else if (unit_of(items, nxt, NH, B, H, nclasses).bh < 0)
-          nxt = claim();
+        const int nxt = valid((int)gridDim.x + __shfl_sync(0xffffffffu, ticket, 0));
         if (ok && cnt > 1) ok = issue_q(1);
         // the following unit's K, V as soon as unit n - 1 has released their
         // buffer: by now its last tiles have passed through the ring

@@ -61,6 +61,7 @@ void free_device(st_layout* L) {
   cudaFree(L->dev.key_ents);
   cudaFree(L->dev.bwd_items);
   for (int f = 1; f < 3; ++f) cudaFree(L->dev.bwd_split[f]);
+  cudaFree(L->dev.sched_slots);
   cudaFree(L->dev.q_ents);
   for (int hc = 0; hc < 2; ++hc)
     for (int k = 0; k < N_ROWLISTS; ++k) cudaFree(L->dev.rows[hc][k]);
@@ -185,6 +186,11 @@ st_status st_pattern_layout(const st_pattern_desc* desc, st_layout** out, void* 
     L->dev.max_split_len[f] = v.empty() ? 0 : v.front().qend - v.front().qbeg;
   }
   L->dev.q_ents_total = (int64_t)L->q_ents.size();
+  if (e == cudaSuccess)
+    e = cudaMalloc(reinterpret_cast<void**>(&L->dev.sched_slots),
+                   2 * kSchedSlots * sizeof(int32_t));
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(L->dev.sched_slots, 0, 2 * kSchedSlots * sizeof(int32_t), cs);
   for (int hc = 0; hc < (int)L->hcs.size() && e == cudaSuccess; ++hc)
     for (int k = 0; k < N_ROWLISTS && e == cudaSuccess; ++k) {
       e = upload(&L->dev.rows[hc][k], L->rows[hc][k], cs);

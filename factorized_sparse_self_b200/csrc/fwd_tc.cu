@@ -8,11 +8,14 @@
 //
 // Persistent CTAs, two per SM (96 KB shared memory and 256 TMEM columns
 // each, so the two CTAs of an SM interleave their MMA and softmax phases).
-// A CTA walks a strided share of the work units (query tile x head, longest
-// first). Warp roles:
-//   warp 4       TMA producer: each unit's Q tile into one of two Q buffers
-//                (the next unit's Q loads while the current one computes)
-//                and K tiles into a 2-stage ring released by the S MMA;
+// Work units (query tile x head, longest first) are claimed from a counter
+// by warp 4 and published to the other roles through a shared-memory ring,
+// so a CTA takes the next unit when it is ready for one. The counter is one
+// of the layout's slots; the last CTA to finish resets it. Warp roles:
+//   warp 4       TMA producer: claims the units; each unit's Q tile into one
+//                of two Q buffers (the next unit's Q loads while the current
+//                one computes) and K tiles into a 2-stage ring released by the
+//                S MMA;
 //   warp 6       TMA producer: V tiles into a 2-stage ring released by PV
 //                (natural, summary or residue-class view for both);
 //   warp 5       TMEM owner and MMA issuer: S = Q K^T (M=128, N=128, K=64)
@@ -39,9 +42,10 @@ namespace {
 using namespace tc;
 
 constexpr int NS = 2;                       // K/V stages
+constexpr int kSched = 4;                   // published work units in flight
 constexpr int kTileBytes = kTile * 64 * 2;  // one 128 x 64 bf16 tile
 constexpr int kThreads = 256;  // warpgroup 0: softmax; warpgroup 1: TMA, MMA
-constexpr uint32_t kRegsSoftmax = 216, kRegsIssue = 40;
+constexpr uint32_t kRegsSoftmax = 208, kRegsIssue = 48;
 static_assert(128 * kRegsSoftmax + 128 * kRegsIssue == kThreads * 128, "register split");
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
@@ -57,6 +61,8 @@ struct SmemFwd {
   uint8_t v[NS][kTileBytes];
   uint64_t q_full[2], q_empty[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   uint64_t s_full, s_free, p_full, pv_done, o_free, fin;
+  uint64_t sched_full[kSched], sched_empty[kSched];
+  int sched[kSched];  // work unit of each slot (n_units: no more work)
   uint32_t tmem_base;
   int abort;
 };
@@ -145,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __restrict__ items,
               int n_units, int NH, const KeyEnt* __restrict__ keys, int B, int H, int nclasses,
               float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-              int* status, uint64_t wait_ns, int force_timeout) {
+              int* sched_slot, int* status, uint64_t wait_ns, int force_timeout) {
   extern __shared__ uint8_t smem_raw[];
   SmemFwd& S = *reinterpret_cast<SmemFwd*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -169,6 +175,10 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
     mbar_init(&S.pv_done, 1);
     mbar_init(&S.o_free, 128);
     mbar_init(&S.fin, 1);
+    for (int k = 0; k < kSched; ++k) {
+      mbar_init(&S.sched_full[k], 1);
+      mbar_init(&S.sched_empty[k], 6);  // V producer, MMA lane, 4 softmax warps
+    }
     S.abort = 0;
     fence_mbar_init();
   }
@@ -182,6 +192,16 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
   auto fail = [&]() {
     *abort = 1;
     set_status(status, ST_ERR_DEVICE_TIMEOUT);
+  };
+  // Next published unit for a consuming role (one arrival per consuming warp).
+  int sk = 0;
+  auto next_unit = [&](int& u, bool arrive) -> bool {
+    const int k = sk % kSched;
+    if (!mbar_wait(&S.sched_full[k], (sk / kSched) & 1, wait_ns, abort)) return false;
+    u = *reinterpret_cast<volatile int*>(&S.sched[k]);
+    if (arrive) mbar_arrive(&S.sched_empty[k]);
+    ++sk;
+    return true;
   };
 
   // Registers: the launch gives 128 per thread; the softmax warpgroup raises
@@ -197,10 +217,33 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       int q_last[2] = {-1, -1};
       int gt = 0;  // global tile counter of this CTA
       bool ok = true;
-      int n = 0;
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-        const Unit x = unit_of(items, u, NH, B, H, nclasses);
-        if (x.bh < 0) continue;
+      int n = 0, pub = 0;
+      // Unit u of the CTA's first is blockIdx.x (the longest units spread one
+      // per CTA); later ones come from the counter, offset by the grid.
+      auto valid = [&](int u) -> int {
+        for (;;) {
+          if (u >= n_units) return n_units;
+          if (unit_of(items, u, NH, B, H, nclasses).bh >= 0) return u;
+          u = (int)gridDim.x + atomicAdd(sched_slot, 1);
+        }
+      };
+      auto publish = [&](int u) -> bool {
+        const int k = pub % kSched;
+        if (!mbar_wait(&S.sched_empty[k], ((pub / kSched) & 1) ^ 1, wait_ns, abort)) return false;
+        S.sched[k] = u;
+        mbar_arrive(&S.sched_full[k]);
+        ++pub;
+        return true;
+      };
+      int cur = valid(blockIdx.x);
+      while (ok && cur < n_units) {
+        if (!publish(cur)) {
+          ok = false;
+          break;
+        }
+        // the claim of the following unit goes out now, answered by the end
+        const int ticket = (int)gridDim.x + atomicAdd(sched_slot, 1);
+        const Unit x = unit_of(items, cur, NH, B, H, nclasses);
         const int qb = n & 1;
         if (!mbar_wait(&S.q_empty[qb], ((n >> 1) & 1) ^ 1, wait_ns, abort)) {
           ok = false;
@@ -226,7 +269,9 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           kv_last[s] = gt;
         }
         ++n;
+        cur = valid(ticket);
       }
+      if (ok && !publish(n_units)) ok = false;  // no more work
       if (!ok) fail();
       // no copy may be in flight when the CTA exits
       for (int b = 0; b < 2; ++b)
@@ -242,9 +287,14 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       int v_last[NS] = {-1, -1};
       int gt = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      for (;;) {
+        int u = 0;
+        if (!next_unit(u, true)) {
+          ok = false;
+          break;
+        }
+        if (u >= n_units) break;
         const Unit x = unit_of(items, u, NH, B, H, nclasses);
-        if (x.bh < 0) continue;
         for (int e = x.it.kbeg; e < x.it.kend; ++e, ++gt) {
           const int s = gt % NS;
           if (!mbar_wait(&S.v_empty[s], ((gt / NS) & 1) ^ 1, wait_ns, abort)) {
@@ -287,16 +337,10 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         mma_commit(&S.k_empty[s]);
         return true;
       };
-      // first unit at or after u with a valid head
-      auto seek = [&](int u, Unit& x) -> int {
-        for (; u < n_units; u += gridDim.x) {
-          x = unit_of(items, u, NH, B, H, nclasses);
-          if (x.bh >= 0) return u;
-        }
-        return n_units;
-      };
-      Unit cur;
-      int u = seek(blockIdx.x, cur);
+      Unit cur, nx;
+      int u = n_units, un = n_units;
+      ok = next_unit(u, true);
+      if (ok && u < n_units) cur = unit_of(items, u, NH, B, H, nclasses);
       bool first_done = false;  // S of this unit's first tile already issued ahead
       while (ok && u < n_units) {
         const int qb = n & 1;
@@ -316,10 +360,20 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           }
         }
         first_done = false;
-        Unit nx;
-        const int un = seek(u + gridDim.x, nx);
+        bool have_next = false;  // the following unit has been read from the ring
         for (int e = 0; e < cnt; ++e, ++gt) {
           const int s = gt % NS;
+          // The following unit is read from the ring at this unit's last tile:
+          // by then all of this unit's K tiles have been issued, so the
+          // producer has published it.
+          if (e + 1 == cnt) {
+            if (!next_unit(un, true)) {
+              ok = false;
+              break;
+            }
+            have_next = true;
+            if (un < n_units) nx = unit_of(items, un, NH, B, H, nclasses);
+          }
           // S of the next tile (this unit's, or the first of the next unit) goes
           // out as soon as the softmax has read S of this one, ahead of PV.
           const bool next_here = (e + 1 < cnt);
@@ -365,6 +419,13 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           mma_commit(&S.v_empty[s]);
         }
         if (!ok) break;
+        if (!have_next) {  // a unit without tiles
+          if (!next_unit(un, true)) {
+            ok = false;
+            break;
+          }
+          if (un < n_units) nx = unit_of(items, un, NH, B, H, nclasses);
+        }
         mma_commit(&S.q_empty[qb]);
         ++n;
         u = un;
@@ -392,8 +453,8 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
     };
     Pending pend = {-1, 0, 0, 0, 0.f, 0.f};
     bool pending = false;
-    auto epilogue = [&](const Pending& pe) {
-      float o[64];
+    // part 1: O out of TMEM (then the accumulator is free for the next unit)
+    auto load_o = [&](const Pending& pe, float* o) {
 #pragma unroll
       for (int xk = 0; xk < 64; ++xk) o[xk] = 0.f;
       if (pe.cnt > 0) {
@@ -403,6 +464,9 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       }
       tc_fence_before();
       mbar_arrive(&S.o_free);
+    };
+    // part 2: normalise, merge with a previous pass, store O and LSE
+    auto finish_o = [&](const Pending& pe, float* o) {
       if (pe.i < 0) return;
       const float inv = (pe.l > 0.f) ? 1.f / pe.l : 0.f;
       float L = (pe.l > 0.f) ? (pe.m + __log2f(pe.l)) * 0.69314718055994531f : -INFINITY;
@@ -440,9 +504,22 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
                              pack_bf16(o[ch * 8 + 6], o[ch * 8 + 7]));
       lse[(size_t)pe.bh * g.T + pe.i] = L;
     };
-    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+    auto epilogue = [&](const Pending& pe) {
+      float o[64];
+      load_o(pe, o);
+      finish_o(pe, o);
+    };
+    for (;;) {
+      int u = 0;
+      const bool got = next_unit(u, false);
+      __syncwarp();
+      if (lane == 0 && got) mbar_arrive(&S.sched_empty[(sk - 1) % kSched]);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      if (u >= n_units) break;
       const Unit x = unit_of(items, u, NH, B, H, nclasses);
-      if (x.bh < 0) continue;
       const FwdItem& it = x.it;
       const int bh = x.bh;
       const int i = view_pos(g, it.qview, it.qtile, row);
@@ -524,10 +601,6 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           if (!ok) break;
           tc_fence_after();
         }
-        if (e == 0 && pending) {
-          epilogue(pend);
-          pending = false;
-        }
         if (__any_sync(0xffffffffu, rescale_o)) {
           const float a = rescale_o ? alpha : 1.f;
 #pragma unroll 1
@@ -543,8 +616,19 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         tmem_st32(tmem + tl + kColP, pk);
         tmem_st32(tmem + tl + kColP + 32, pk + 32);
         tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&S.p_full);
+        // the previous unit's O leaves TMEM before this unit's first PV may
+        // start; its normalisation and stores overlap that PV
+        if (e == 0 && pending) {
+          float o[64];
+          load_o(pend, o);
+          tc_fence_before();
+          mbar_arrive(&S.p_full);
+          finish_o(pend, o);
+          pending = false;
+        } else {
+          tc_fence_before();
+          mbar_arrive(&S.p_full);
+        }
       }
       if (!ok) break;
       pend = {i, bh, cnt, (int)it.merge, m_run, l_run};
@@ -563,6 +647,14 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
   tc_fence_before();
   __syncthreads();
   if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+  // the last CTA out resets the work counter for the slot's next launch
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(sched_slot + 1, 1) == (int)gridDim.x - 1) {
+      atomicExch(sched_slot, 0);
+      atomicExch(sched_slot + 1, 0);
+    }
+  }
 }
 
 }  // namespace
@@ -590,6 +682,7 @@ cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, v
   const int sms = sm_count();
   const float scale_log2 = c.scale * 1.4426950408889634f;
   const int NH = heads_per_class(c);
+  int* slot = L->dev.sched_slots + 2 * (L->next_slot.fetch_add(1) % kSchedSlots);
   record_begin(c);
   for (int pass = 0; pass < L->n_passes; ++pass) {
     const int n = L->dev.n_fwd_items[pass];
@@ -600,7 +693,7 @@ cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, v
     fwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
         maps, L->geom, (const FwdItem*)L->dev.fwd_items[pass], (int)units, NH,
         (const KeyEnt*)L->dev.key_ents, c.B, c.H, c.nclasses, scale_log2, (__nv_bfloat16*)o, lse,
-        c.status, c.wait_ns, (force_timeout && pass == 0) ? 1 : 0);
+        slot, c.status, c.wait_ns, (force_timeout && pass == 0) ? 1 : 0);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }

@@ -2,6 +2,7 @@
 // of libsparse_transformer_attn.so. Not part of the public ABI.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <vector>
 
@@ -11,6 +12,7 @@ namespace st {
 
 constexpr int kTile = 128;  // query and key tile edge, in view rows
 constexpr int kBwdChunk = 8; // most query tiles one backward work item visits
+constexpr int kSchedSlots = 64;  // forward calls of one layout that may run at once
 
 // Row orders ("views") a segment reads its queries or keys in.
 enum View : uint8_t {
@@ -121,6 +123,9 @@ struct DeviceSchedule {
   int32_t n_bwd_split[3] = {0, 0, 0};
   int32_t max_split_len[3] = {0, 0, 0};  // most query tiles of one item
   int64_t q_ents_total = 0;
+  // work counters of the forward kernel: kSchedSlots pairs (next unit, CTAs
+  // done), zero between launches (the last CTA of a launch resets its pair)
+  int32_t* sched_slots = nullptr;
   void* q_ents = nullptr;
   int32_t max_fwd_keys = 0;    // longest key list of a forward item
   // per head class (at most 2) and row list: device array of natural rows
@@ -146,6 +151,7 @@ struct st_layout {
   std::vector<int32_t> rows[2][st::N_ROWLISTS];  // see st::RowList
   bool on_device = false;
   int device = -1;
+  mutable std::atomic<uint32_t> next_slot{0};  // round robin over dev.sched_slots
   st::DeviceSchedule dev;
 };
 
