@@ -131,7 +131,10 @@ st_status st_layout_nnz(const st_layout* layout, int32_t head_class, int64_t* nn
  * [B, H, T, d] tensors (split mode picks A1/A2 from its parity). Rows with an
  * empty set get O = 0 and LSE = -inf. For a strided merged layout the call
  * runs two passes (natural-order window keys, then residue-order strided
- * keys) and merges them by log-sum-exp in place in o and lse. */
+ * keys) and merges them by log-sum-exp in place in o and lse. On the bf16
+ * path each call takes one of the layout's 64 work counters in turn: at most
+ * 64 forward calls of one layout may be in flight at the same time (on
+ * different streams, or in concurrently replayed graphs). */
 st_status st_sparse_attn_fwd(const st_layout* layout, st_dtype dtype, int32_t B, int32_t H,
                              int32_t T, int32_t d, float scale, const void* q, const void* k,
                              const void* v, void* o, float* lse, void* stream);
