@@ -43,6 +43,11 @@ SIGNATURES = {
     "st_sparse_attn_bwd": (ctypes.c_int, [_P, ctypes.c_int, _i32, _i32, _i32, _i32,
                                           ctypes.c_float, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                           _P, ctypes.c_size_t, _P]),
+    "st_sparse_attn_fwd_heads": (ctypes.c_int, [_P, ctypes.c_int, _i32, _i32, _i32, _i32, _i32,
+                                                _i32, ctypes.c_float, _P, _P, _P, _P, _P, _P]),
+    "st_sparse_attn_bwd_heads": (ctypes.c_int, [_P, ctypes.c_int, _i32, _i32, _i32, _i32, _i32,
+                                                _i32, ctypes.c_float, _P, _P, _P, _P, _P, _P, _P,
+                                                _P, _P, _P, ctypes.c_size_t, _P]),
     "st_sparse_attn_bwd_noalloc": (ctypes.c_int, [_P, ctypes.c_int, _i32, _i32, _i32, _i32,
                                                   ctypes.c_float, _P, _P, _P, _P, _P, _P, _P, _P,
                                                   _P, _P]),
@@ -194,8 +199,11 @@ def _need(t, name, like=None):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def st_sparse_attn_fwd(layout: Layout, q, k, v, scale=None, o=None, lse=None, stream=None):
-    """O [B,H,T,d] (dtype of q) and LSE [B,H,T] float32 for all heads."""
+def st_sparse_attn_fwd(layout: Layout, q, k, v, scale=None, o=None, lse=None, stream=None,
+                       heads=None):
+    """O [B,H,T,d] (dtype of q) and LSE [B,H,T] float32 for all heads, or for
+    heads = (begin, count) only (st_sparse_attn_fwd_heads; other heads' rows
+    of o and lse are left as they are)."""
     import torch
     B, H, T, d = q.shape
     if o is None:
@@ -203,10 +211,17 @@ def st_sparse_attn_fwd(layout: Layout, q, k, v, scale=None, o=None, lse=None, st
     if lse is None:
         lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
     args = [_need(x, n, q) for x, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"))]
-    code = lib().st_sparse_attn_fwd(layout.handle, _dtype_code(q), B, H, T, d,
-                                    float(scale) if scale else 0.0, args[0], args[1], args[2],
-                                    args[3], _need(lse, "lse"), _stream_ptr(stream))
-    _check(code, "st_sparse_attn_fwd")
+    sc = float(scale) if scale else 0.0
+    if heads is None:
+        code = lib().st_sparse_attn_fwd(layout.handle, _dtype_code(q), B, H, T, d, sc, args[0],
+                                        args[1], args[2], args[3], _need(lse, "lse"),
+                                        _stream_ptr(stream))
+        _check(code, "st_sparse_attn_fwd")
+    else:
+        code = lib().st_sparse_attn_fwd_heads(layout.handle, _dtype_code(q), B, H, heads[0],
+                                              heads[1], T, d, sc, args[0], args[1], args[2],
+                                              args[3], _need(lse, "lse"), _stream_ptr(stream))
+        _check(code, "st_sparse_attn_fwd_heads")
     return o, lse
 
 
@@ -218,8 +233,9 @@ def st_sparse_attn_bwd_workspace(layout: Layout, dtype, B, H, T, d) -> int:
 
 
 def st_sparse_attn_bwd(layout: Layout, q, k, v, o, lse, dout, scale=None, workspace=None,
-                       dq=None, dk=None, dv=None, stream=None):
-    """dQ, dK, dV (dtype of q), with P recomputed from LSE."""
+                       dq=None, dk=None, dv=None, stream=None, heads=None):
+    """dQ, dK, dV (dtype of q), with P recomputed from LSE; for heads =
+    (begin, count) only when given (st_sparse_attn_bwd_heads)."""
     import torch
     B, H, T, d = q.shape
     if workspace is None:
@@ -230,12 +246,21 @@ def st_sparse_attn_bwd(layout: Layout, q, k, v, o, lse, dout, scale=None, worksp
     dv = torch.empty_like(q) if dv is None else dv
     ptrs = [_need(x, n, q) for x, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"),
                                         (dq, "dq"), (dk, "dk"), (dv, "dv"))]
-    code = lib().st_sparse_attn_bwd(layout.handle, _dtype_code(q), B, H, T, d,
-                                    float(scale) if scale else 0.0, ptrs[0], ptrs[1], ptrs[2],
-                                    ptrs[3], _need(lse, "lse"), ptrs[4], ptrs[5], ptrs[6], ptrs[7],
-                                    ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
-                                    _stream_ptr(stream))
-    _check(code, "st_sparse_attn_bwd")
+    sc = float(scale) if scale else 0.0
+    ws = ctypes.c_void_p(workspace.data_ptr())
+    if heads is None:
+        code = lib().st_sparse_attn_bwd(layout.handle, _dtype_code(q), B, H, T, d, sc, ptrs[0],
+                                        ptrs[1], ptrs[2], ptrs[3], _need(lse, "lse"), ptrs[4],
+                                        ptrs[5], ptrs[6], ptrs[7], ws, workspace.numel(),
+                                        _stream_ptr(stream))
+        _check(code, "st_sparse_attn_bwd")
+    else:
+        code = lib().st_sparse_attn_bwd_heads(layout.handle, _dtype_code(q), B, H, heads[0],
+                                              heads[1], T, d, sc, ptrs[0], ptrs[1], ptrs[2],
+                                              ptrs[3], _need(lse, "lse"), ptrs[4], ptrs[5],
+                                              ptrs[6], ptrs[7], ws, workspace.numel(),
+                                              _stream_ptr(stream))
+        _check(code, "st_sparse_attn_bwd_heads")
     return dq, dk, dv
 
 

@@ -187,17 +187,16 @@ struct Unit {
   int bh;
 };
 
-__device__ __forceinline__ Unit unit_of(const BwdItem* items, int u, int NH, int B, int H,
-                                        int nclasses) {
+__device__ __forceinline__ Unit unit_of(const BwdItem* items, int u, int NH, const Heads& hs) {
   Unit x;
   x.it = items[u / NH];
-  x.bh = head_of(u % NH, x.it.hclass, B, H, nclasses);
+  x.bh = head_of(u % NH, x.it.hclass, hs);
   return x;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __restrict__ items,
-              int n_units, int NH, const QEnt* __restrict__ qents, int B, int H, int nclasses,
+              int n_units, int NH, const QEnt* __restrict__ qents, Heads hs,
               float scale, float scale_log2, const float* __restrict__ lse,
               const float* __restrict__ Dg, int* sched_counter, int* status,
               uint64_t wait_ns) {
@@ -281,7 +280,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       auto valid = [&](int u) -> int {
         for (;;) {
           if (u >= n_units) return n_units;
-          if (unit_of(items, u, NH, B, H, nclasses).bh >= 0) return u;
+          if (unit_of(items, u, NH, hs).bh >= 0) return u;
           int t = 0;
           if (lane == 0) t = atomicAdd(sched_counter, 1);
           u = (int)gridDim.x + __shfl_sync(0xffffffffu, t, 0);
@@ -306,7 +305,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         // needed once this unit's K, V are on their way
         int ticket = 0;
         if (lane == 0) ticket = atomicAdd(sched_counter, 1);
-        const Unit x = unit_of(items, cur, NH, B, H, nclasses);
+        const Unit x = unit_of(items, cur, NH, hs);
         const int cnt = x.it.qend - x.it.qbeg;
         auto issue_q = [&](int e) -> bool {
           const int s = gt % NS;
@@ -369,7 +368,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         if (ok && cnt > 1) ok = issue_q(1);
         // the following unit's K, V as soon as unit n - 1 has released their
         // buffer: by now its last tiles have passed through the ring
-        if (ok && nxt < n_units) ok = load_kv(n + 1, unit_of(items, nxt, NH, B, H, nclasses));
+        if (ok && nxt < n_units) ok = load_kv(n + 1, unit_of(items, nxt, NH, hs));
         for (int e = 2; ok && e < cnt; ++e) ok = issue_q(e);
         ++n;
         cur = nxt;
@@ -419,7 +418,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             break;
           }
           if (u >= n_units) break;
-          const Unit x = unit_of(items, u, NH, B, H, nclasses);
+          const Unit x = unit_of(items, u, NH, hs);
           const int cnt = x.it.qend - x.it.qbeg;
           const int kb = n & 1;
           k_addr = smem_u32(S.k[kb]);
@@ -505,7 +504,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             break;
           }
           if (u >= n_units) break;
-          const Unit x = unit_of(items, u, NH, B, H, nclasses);
+          const Unit x = unit_of(items, u, NH, hs);
           const int cnt = x.it.qend - x.it.qbeg;
           for (int e = 0; ok && e < cnt; ++e, ++gt) {
             if (gt > 0 && !reduce_dq(gt - 1)) {
@@ -594,7 +593,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         break;
       }
       if (u >= n_units) break;
-      const Unit x = unit_of(items, u, NH, B, H, nclasses);
+      const Unit x = unit_of(items, u, NH, hs);
       const BwdItem& it = x.it;
       const int cnt = it.qend - it.qbeg;
       const int j = view_pos(g, it.kview, it.ktile, row);
@@ -770,7 +769,7 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, c
   record_begin(c);
   bwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
       maps, L->geom, (const BwdItem*)L->dev.bwd_split[f], (int)units, NH,
-      (const QEnt*)L->dev.q_ents, c.B, c.H, c.nclasses, c.scale, c.scale * kLog2e, lse, D,
+      (const QEnt*)L->dev.q_ents, heads_of(c), c.scale, c.scale * kLog2e, lse, D,
       sched_counter, c.status,
       c.wait_ns);
   err = cudaGetLastError();

@@ -72,11 +72,12 @@ void free_device(st_layout* L) {
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Common checks of fwd / bwd. Returns ST_OK and fills the call on success.
-st_status prepare(const st_layout* L, st_dtype dtype, int32_t B, int32_t H, int32_t T, int32_t d,
-                  float scale, void* stream, Call& c) {
+st_status prepare(const st_layout* L, st_dtype dtype, int32_t B, int32_t H, int32_t h0, int32_t hn,
+                  int32_t T, int32_t d, float scale, void* stream, Call& c) {
   if (!L || !L->on_device) return ST_ERR_INVALID;
   if (dtype != ST_F32 && dtype != ST_BF16) return ST_ERR_INVALID;
   if (B < 1 || H < 1 || d < 1 || T != L->geom.T) return ST_ERR_INVALID;
+  if (h0 < 0 || hn < 1 || (int64_t)h0 + hn > H) return ST_ERR_INVALID;
   if ((int64_t)B * H > (1 << 30) || (int64_t)B * H * T * d > (int64_t)1 << 40) return ST_ERR_INVALID;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return ST_ERR_CUDA;
@@ -88,8 +89,7 @@ st_status prepare(const st_layout* L, st_dtype dtype, int32_t B, int32_t H, int3
     if (T % kTile != 0 || !L->tc_ok) return ST_ERR_UNSUPPORTED;
   }
   int nclasses = (int)L->hcs.size();
-  int per = nclasses == 1 ? B * H : B * ((H + 1) / 2);
-  if (per > 2147483647 / 2) return ST_ERR_UNSUPPORTED;
+  if ((int64_t)B * hn > 2147483647 / 2) return ST_ERR_UNSUPPORTED;
   for (int p = 0; p < L->n_passes; ++p)
     if (L->dev.n_fwd_items[p] > 65535) return ST_ERR_UNSUPPORTED;
   if (L->dev.n_bwd_items > 65535) return ST_ERR_UNSUPPORTED;
@@ -97,6 +97,8 @@ st_status prepare(const st_layout* L, st_dtype dtype, int32_t B, int32_t H, int3
   c.dtype = dtype;
   c.B = B;
   c.H = H;
+  c.h0 = h0;
+  c.hn = hn;
   c.d = d;
   c.scale = (scale > 0.f) ? scale : 1.0f / sqrtf((float)d);
   c.nclasses = nclasses;
@@ -283,8 +285,15 @@ st_status st_layout_export(const st_layout* L, int32_t hc, int32_t seg, int32_t 
 st_status st_sparse_attn_fwd(const st_layout* L, st_dtype dtype, int32_t B, int32_t H, int32_t T,
                              int32_t d, float scale, const void* q, const void* k, const void* v,
                              void* o, float* lse, void* stream) {
+  return st_sparse_attn_fwd_heads(L, dtype, B, H, 0, H, T, d, scale, q, k, v, o, lse, stream);
+}
+
+st_status st_sparse_attn_fwd_heads(const st_layout* L, st_dtype dtype, int32_t B, int32_t H,
+                                   int32_t h_begin, int32_t h_count, int32_t T, int32_t d,
+                                   float scale, const void* q, const void* k, const void* v,
+                                   void* o, float* lse, void* stream) {
   Call c;
-  st_status s = prepare(L, dtype, B, H, T, d, scale, stream, c);
+  st_status s = prepare(L, dtype, B, H, h_begin, h_count, T, d, scale, stream, c);
   if (s != ST_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return ST_ERR_INVALID;
@@ -315,8 +324,18 @@ st_status st_sparse_attn_bwd(const st_layout* L, st_dtype dtype, int32_t B, int3
                              int32_t d, float scale, const void* q, const void* k, const void* v,
                              const void* o, const float* lse, const void* dout, void* dq,
                              void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream) {
+  return st_sparse_attn_bwd_heads(L, dtype, B, H, 0, H, T, d, scale, q, k, v, o, lse, dout, dq,
+                                  dk, dv, workspace, ws_bytes, stream);
+}
+
+st_status st_sparse_attn_bwd_heads(const st_layout* L, st_dtype dtype, int32_t B, int32_t H,
+                                   int32_t h_begin, int32_t h_count, int32_t T, int32_t d,
+                                   float scale, const void* q, const void* k, const void* v,
+                                   const void* o, const float* lse, const void* dout, void* dq,
+                                   void* dk, void* dv, void* workspace, size_t ws_bytes,
+                                   void* stream) {
   Call c;
-  st_status s = prepare(L, dtype, B, H, T, d, scale, stream, c);
+  st_status s = prepare(L, dtype, B, H, h_begin, h_count, T, d, scale, stream, c);
   if (s != ST_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
@@ -330,9 +349,13 @@ st_status st_sparse_attn_bwd(const st_layout* L, st_dtype dtype, int32_t B, int3
   float* Dv = reinterpret_cast<float*>(workspace);
   cudaError_t e;
   if (dtype == ST_F32) {
-    e = cudaMemsetAsync(dq, 0, elems * sizeof(float), c.stream);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, elems * sizeof(float), c.stream);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, elems * sizeof(float), c.stream);
+    // the selected heads of every batch: B rows of hn*T*d floats, H*T*d apart
+    const size_t head = (size_t)T * d * sizeof(float);
+    void* outs[3] = {dq, dk, dv};
+    e = cudaSuccess;
+    for (int x = 0; x < 3 && e == cudaSuccess; ++x)
+      e = cudaMemset2DAsync(static_cast<char*>(outs[x]) + (size_t)c.h0 * head, (size_t)H * head, 0,
+                            (size_t)c.hn * head, (size_t)B, c.stream);
     if (e == cudaSuccess) e = bwd_prologue(c, o, dout, Dv, nullptr, 0);
     Call cm = c;
     arm(cm, 1);

@@ -55,12 +55,27 @@ __device__ __forceinline__ bool rule_live(const Geom& g, int rule, int i, int j)
 
 // Head index bh = b*H + h of grid column x for a head class: split mode puts
 // even heads in class 0 and odd heads in class 1. Returns -1 past the end.
-__device__ __forceinline__ int head_of(int x, int hclass, int B, int H, int nclasses) {
-  if (nclasses == 1) return x < B * H ? x : -1;
-  int per = (hclass == 0) ? (H + 1) / 2 : H / 2;
-  if (per == 0 || x >= B * per) return -1;
-  int b = x / per, hh = x - b * per;
-  return b * H + 2 * hh + hclass;
+// Flat index of the x-th head of class hclass among the heads h0 .. h0+hn-1
+// of a [B, H, T, d] tensor, or -1 past the end. Split layouts give class p
+// the heads of parity p (global head index, so a head range keeps each head's
+// set); merged layouts have one class.
+__device__ __forceinline__ int head_of(int x, int hclass, const Heads& hs) {
+  if (hs.nclasses == 1) {
+    if (x >= hs.B * hs.hn) return -1;
+    const int b = x / hs.hn;
+    return b * hs.H + hs.h0 + (x - b * hs.hn);
+  }
+  const int first = hs.h0 + ((hclass - hs.h0) & 1);
+  const int end = hs.h0 + hs.hn;
+  const int per = first < end ? (end - 1 - first) / 2 + 1 : 0;
+  if (per == 0 || x >= hs.B * per) return -1;
+  const int b = x / per;
+  return b * hs.H + first + 2 * (x - b * per);
+}
+
+// Head class of flat head index bh (0 for merged layouts).
+__device__ __forceinline__ int class_of(int bh, const Heads& hs) {
+  return hs.nclasses == 2 ? ((bh % hs.H) & 1) : 0;
 }
 
 __device__ __forceinline__ void set_status(int* status, int code) {

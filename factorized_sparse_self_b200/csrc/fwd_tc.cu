@@ -139,17 +139,16 @@ struct Unit {
   int bh;
 };
 
-__device__ __forceinline__ Unit unit_of(const FwdItem* items, int u, int NH, int B, int H,
-                                        int nclasses) {
+__device__ __forceinline__ Unit unit_of(const FwdItem* items, int u, int NH, const Heads& hs) {
   Unit x;
   x.it = items[u / NH];
-  x.bh = head_of(u % NH, x.it.hclass, B, H, nclasses);
+  x.bh = head_of(u % NH, x.it.hclass, hs);
   return x;
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
 fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __restrict__ items,
-              int n_units, int NH, const KeyEnt* __restrict__ keys, int B, int H, int nclasses,
+              int n_units, int NH, const KeyEnt* __restrict__ keys, Heads hs,
               float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
               int* sched_slot, int* status, uint64_t wait_ns, int force_timeout) {
   extern __shared__ uint8_t smem_raw[];
@@ -223,7 +222,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       auto valid = [&](int u) -> int {
         for (;;) {
           if (u >= n_units) return n_units;
-          if (unit_of(items, u, NH, B, H, nclasses).bh >= 0) return u;
+          if (unit_of(items, u, NH, hs).bh >= 0) return u;
           u = (int)gridDim.x + atomicAdd(sched_slot, 1);
         }
       };
@@ -243,7 +242,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         }
         // the claim of the following unit goes out now, answered by the end
         const int ticket = (int)gridDim.x + atomicAdd(sched_slot, 1);
-        const Unit x = unit_of(items, cur, NH, B, H, nclasses);
+        const Unit x = unit_of(items, cur, NH, hs);
         const int qb = n & 1;
         if (!mbar_wait(&S.q_empty[qb], ((n >> 1) & 1) ^ 1, wait_ns, abort)) {
           ok = false;
@@ -294,7 +293,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           break;
         }
         if (u >= n_units) break;
-        const Unit x = unit_of(items, u, NH, B, H, nclasses);
+        const Unit x = unit_of(items, u, NH, hs);
         for (int e = x.it.kbeg; e < x.it.kend; ++e, ++gt) {
           const int s = gt % NS;
           if (!mbar_wait(&S.v_empty[s], ((gt / NS) & 1) ^ 1, wait_ns, abort)) {
@@ -340,7 +339,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       Unit cur, nx;
       int u = n_units, un = n_units;
       ok = next_unit(u, true);
-      if (ok && u < n_units) cur = unit_of(items, u, NH, B, H, nclasses);
+      if (ok && u < n_units) cur = unit_of(items, u, NH, hs);
       bool first_done = false;  // S of this unit's first tile already issued ahead
       while (ok && u < n_units) {
         const int qb = n & 1;
@@ -372,7 +371,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
               break;
             }
             have_next = true;
-            if (un < n_units) nx = unit_of(items, un, NH, B, H, nclasses);
+            if (un < n_units) nx = unit_of(items, un, NH, hs);
           }
           // S of the next tile (this unit's, or the first of the next unit) goes
           // out as soon as the softmax has read S of this one, ahead of PV.
@@ -424,7 +423,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
             ok = false;
             break;
           }
-          if (un < n_units) nx = unit_of(items, un, NH, B, H, nclasses);
+          if (un < n_units) nx = unit_of(items, un, NH, hs);
         }
         mma_commit(&S.q_empty[qb]);
         ++n;
@@ -519,7 +518,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         break;
       }
       if (u >= n_units) break;
-      const Unit x = unit_of(items, u, NH, B, H, nclasses);
+      const Unit x = unit_of(items, u, NH, hs);
       const FwdItem& it = x.it;
       const int bh = x.bh;
       const int i = view_pos(g, it.qview, it.qtile, row);
@@ -692,7 +691,7 @@ cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, v
     const int grid = (int)std::min<long long>(units, 2LL * sms);
     fwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
         maps, L->geom, (const FwdItem*)L->dev.fwd_items[pass], (int)units, NH,
-        (const KeyEnt*)L->dev.key_ents, c.B, c.H, c.nclasses, scale_log2, (__nv_bfloat16*)o, lse,
+        (const KeyEnt*)L->dev.key_ents, heads_of(c), scale_log2, (__nv_bfloat16*)o, lse,
         slot, c.status, c.wait_ns, (force_timeout && pass == 0) ? 1 : 0);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;

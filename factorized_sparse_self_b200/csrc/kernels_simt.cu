@@ -35,7 +35,7 @@ __device__ __forceinline__ float dot_smem(const float* a, const float* b) {
 template <class E, int D>
 __global__ void __launch_bounds__(kThreads)
 simt_fwd_kernel(Geom g, const FwdItem* __restrict__ items, const KeyEnt* __restrict__ keys,
-                int B, int H, int nclasses, float scale, const E* __restrict__ q,
+                Heads hs, float scale, const E* __restrict__ q,
                 const E* __restrict__ k, const E* __restrict__ v, E* __restrict__ o,
                 float* __restrict__ lse) {
   extern __shared__ float sm[];
@@ -43,7 +43,7 @@ simt_fwd_kernel(Geom g, const FwdItem* __restrict__ items, const KeyEnt* __restr
   float* Vs = Ks + kTile * (D + 1);
   int* jpos = reinterpret_cast<int*>(Vs + kTile * (D + 1));
   const FwdItem it = items[blockIdx.y];
-  const int bh = head_of(blockIdx.x, it.hclass, B, H, nclasses);
+  const int bh = head_of(blockIdx.x, it.hclass, hs);
   if (bh < 0) return;
   const size_t base = (size_t)bh * g.T * D;
   const int tid = threadIdx.x;
@@ -118,7 +118,7 @@ simt_fwd_kernel(Geom g, const FwdItem* __restrict__ items, const KeyEnt* __restr
 template <class E, int D>
 __global__ void __launch_bounds__(kThreads)
 simt_bwd_kv_kernel(Geom g, const BwdItem* __restrict__ items, const QEnt* __restrict__ qents,
-                   int B, int H, int nclasses, float scale, const E* __restrict__ q,
+                   Heads hs, float scale, const E* __restrict__ q,
                    const E* __restrict__ k, const E* __restrict__ v, const float* __restrict__ lse,
                    const E* __restrict__ dout, const float* __restrict__ Dv,
                    float* __restrict__ dk_acc, float* __restrict__ dv_acc) {
@@ -131,7 +131,7 @@ simt_bwd_kv_kernel(Geom g, const BwdItem* __restrict__ items, const QEnt* __rest
   float* Ds = lses + kTile;
   int* ipos = reinterpret_cast<int*>(Ds + kTile);
   const BwdItem it = items[blockIdx.y];
-  const int bh = head_of(blockIdx.x, it.hclass, B, H, nclasses);
+  const int bh = head_of(blockIdx.x, it.hclass, hs);
   if (bh < 0) return;
   const size_t base = (size_t)bh * g.T * D;
   const size_t rbase = (size_t)bh * g.T;
@@ -194,7 +194,7 @@ simt_bwd_kv_kernel(Geom g, const BwdItem* __restrict__ items, const QEnt* __rest
 template <class E, int D>
 __global__ void __launch_bounds__(kThreads)
 simt_bwd_q_kernel(Geom g, const FwdItem* __restrict__ items, const KeyEnt* __restrict__ keys,
-                  int B, int H, int nclasses, float scale, const E* __restrict__ q,
+                  Heads hs, float scale, const E* __restrict__ q,
                   const E* __restrict__ k, const E* __restrict__ v,
                   const float* __restrict__ lse, const E* __restrict__ dout,
                   const float* __restrict__ Dv, float* __restrict__ dq_acc) {
@@ -206,7 +206,7 @@ simt_bwd_q_kernel(Geom g, const FwdItem* __restrict__ items, const KeyEnt* __res
   int* jpos = reinterpret_cast<int*>(dOo + kTile * (D + 1));
   const FwdItem it = items[blockIdx.y];
   if (it.kbeg == it.kend) return;
-  const int bh = head_of(blockIdx.x, it.hclass, B, H, nclasses);
+  const int bh = head_of(blockIdx.x, it.hclass, hs);
   if (bh < 0) return;
   const size_t base = (size_t)bh * g.T * D;
   const int tid = threadIdx.x;
@@ -312,13 +312,14 @@ __device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
 
 __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
                                 float* __restrict__ Dv,
-                                int T, int H, int nclasses, RowSet rs, float4* __restrict__ dq_acc,
+                                int T, Heads hs, RowSet rs, float4* __restrict__ dq_acc,
                                 float4* __restrict__ dk_acc, float4* __restrict__ dv_acc,
                                 uint4* __restrict__ dq, uint4* __restrict__ dk,
                                 uint4* __restrict__ dv, int* __restrict__ sched_counter) {
-  const int bh = blockIdx.y;
+  // grid.y runs over the selected heads of every batch
+  const int bh = (blockIdx.y / hs.hn) * hs.H + hs.h0 + blockIdx.y % hs.hn;
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *sched_counter = 0;
-  const int hc = (nclasses == 2) ? ((bh % H) & 1) : 0;
+  const int hc = class_of(bh, hs);
   const size_t rb = (size_t)bh * T;
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int stride = gridDim.x * blockDim.x;
@@ -397,11 +398,11 @@ __device__ __forceinline__ uint4 round8f(const float4& a, const float4& b, float
 // per thread and step.
 __global__ void bwd_finish_kernel(const float4* __restrict__ dq_acc,
                                   const float4* __restrict__ dk_acc,
-                                  const float4* __restrict__ dv_acc, int T, int H, int nclasses,
+                                  const float4* __restrict__ dv_acc, int T, Heads hs,
                                   RowSet rs, float scale, uint4* __restrict__ dq,
                                   uint4* __restrict__ dk, uint4* __restrict__ dv) {
-  const int bh = blockIdx.y;
-  const int hc = (nclasses == 2) ? ((bh % H) & 1) : 0;
+  const int bh = (blockIdx.y / hs.hn) * hs.H + hs.h0 + blockIdx.y % hs.hn;
+  const int hc = class_of(bh, hs);
   const size_t rb = (size_t)bh * T;
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int stride = gridDim.x * blockDim.x;
@@ -446,8 +447,8 @@ cudaError_t simt_fwd_t(const Call& c, const void* q, const void* k, const void* 
     if (n == 0) continue;
     dim3 grid(heads_per_class(c), n);
     kern<<<grid, kThreads, smem, c.stream>>>(
-        L->geom, (const FwdItem*)L->dev.fwd_items[pass], (const KeyEnt*)L->dev.key_ents, c.B,
-        c.H, c.nclasses, c.scale, (const E*)q, (const E*)k, (const E*)v, (E*)o, lse);
+        L->geom, (const FwdItem*)L->dev.fwd_items[pass], (const KeyEnt*)L->dev.key_ents,
+        heads_of(c), c.scale, (const E*)q, (const E*)k, (const E*)v, (E*)o, lse);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
@@ -473,8 +474,8 @@ cudaError_t simt_bwd_t(const Call& c, const void* q, const void* k, const void* 
   if (L->dev.n_bwd_items > 0) {
     dim3 grid(heads_per_class(c), L->dev.n_bwd_items);
     kv<<<grid, kThreads, smem_kv, c.stream>>>(
-        L->geom, (const BwdItem*)L->dev.bwd_items, (const QEnt*)L->dev.q_ents, c.B, c.H,
-        c.nclasses, c.scale, (const E*)q, (const E*)k, (const E*)v, lse, (const E*)dout, Dv,
+        L->geom, (const BwdItem*)L->dev.bwd_items, (const QEnt*)L->dev.q_ents,
+        heads_of(c), c.scale, (const E*)q, (const E*)k, (const E*)v, lse, (const E*)dout, Dv,
         dk_acc, dv_acc);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
@@ -484,8 +485,8 @@ cudaError_t simt_bwd_t(const Call& c, const void* q, const void* k, const void* 
     if (n == 0) continue;
     dim3 grid(heads_per_class(c), n);
     kq<<<grid, kThreads, smem_q, c.stream>>>(
-        L->geom, (const FwdItem*)L->dev.fwd_items[pass], (const KeyEnt*)L->dev.key_ents, c.B,
-        c.H, c.nclasses, c.scale, (const E*)q, (const E*)k, (const E*)v, lse, (const E*)dout,
+        L->geom, (const FwdItem*)L->dev.fwd_items[pass], (const KeyEnt*)L->dev.key_ents,
+        heads_of(c), c.scale, (const E*)q, (const E*)k, (const E*)v, lse, (const E*)dout,
         Dv, dq_acc);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
@@ -537,9 +538,9 @@ cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* Dv, 
                      int* sched_counter) {
   const int T = c.L->geom.T;
   const int bx = std::max(1, std::min(64, (T + 127) / 128));
-  dim3 grid(bx, c.B * c.H);
+  dim3 grid(bx, c.B * c.hn);
   bwd_prep_kernel<<<grid, 256, 0, c.stream>>>(
-      (const uint4*)o, (const uint4*)dout, Dv, T, c.H, c.nclasses,
+      (const uint4*)o, (const uint4*)dout, Dv, T, heads_of(c),
       row_set_of(c.L), (float4*)dq_acc, (float4*)dk_acc, (float4*)dv_acc, (uint4*)dq, (uint4*)dk,
       (uint4*)dv, sched_counter);
   return cudaGetLastError();
@@ -553,10 +554,10 @@ cudaError_t bwd_finish(const Call& c, const float* dq_acc, const float* dk_acc,
     most = std::max(most, std::max(L->dev.n_rows[hc][ROWS_Q_ACC], L->dev.n_rows[hc][ROWS_K_ACC]));
   if (most == 0) return cudaSuccess;  // every row was written directly
   const int bx = std::max(1, std::min(64, (most + 31) / 32));
-  dim3 grid(bx, c.B * c.H);
+  dim3 grid(bx, c.B * c.hn);
   bwd_finish_kernel<<<grid, 256, 0, c.stream>>>(
-      (const float4*)dq_acc, (const float4*)dk_acc, (const float4*)dv_acc, L->geom.T, c.H,
-      c.nclasses, row_set_of(L), c.scale, (uint4*)dq, (uint4*)dk, (uint4*)dv);
+      (const float4*)dq_acc, (const float4*)dk_acc, (const float4*)dv_acc, L->geom.T,
+      heads_of(c), row_set_of(L), c.scale, (uint4*)dq, (uint4*)dk, (uint4*)dv);
   return cudaGetLastError();
 }
 

@@ -3,6 +3,8 @@
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "st_internal.h"
 
 namespace st {
@@ -11,6 +13,7 @@ struct Call {
   const st_layout* L;
   int dtype;  // st_dtype
   int B, H, d;
+  int h0 = 0, hn = 0;  // heads h0 .. h0+hn-1 of the H in the tensors
   float scale;
   int nclasses;     // head classes of the layout
   int* status;      // device status word
@@ -69,8 +72,26 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v,
 
 namespace st {
 
+inline Heads heads_of(const Call& c) {
+  Heads h;
+  h.B = c.B;
+  h.H = c.H;
+  h.h0 = c.h0;
+  h.hn = c.hn;
+  h.nclasses = c.nclasses;
+  return h;
+}
+
+// Units per item: the most heads of one class among the selected heads, times B.
 inline int heads_per_class(const Call& c) {
-  return c.nclasses == 1 ? c.B * c.H : c.B * ((c.H + 1) / 2);
+  if (c.nclasses == 1) return c.B * c.hn;
+  int most = 0;
+  for (int p = 0; p < 2; ++p) {
+    const int first = c.h0 + ((p - c.h0) & 1);
+    const int end = c.h0 + c.hn;
+    most = std::max(most, first < end ? (end - 1 - first) / 2 + 1 : 0);
+  }
+  return c.B * most;
 }
 
 // Encodes the natural (3-D), summary and residue-class (4-D) TMA views of a

@@ -84,6 +84,12 @@ enum RowList : int {
   N_ROWLISTS = 4
 };
 
+// Heads a call covers: heads h0 .. h0+hn-1 of tensors with B x H heads, for a
+// layout with nclasses head classes (kernel parameter, plain old data).
+struct Heads {
+  int32_t B, H, h0, hn, nclasses;
+};
+
 // Geometry every kernel needs to map view rows to natural positions.
 struct Geom {
   int32_t T, l, c;

@@ -155,6 +155,27 @@ st_status st_sparse_attn_bwd(const st_layout* layout, st_dtype dtype, int32_t B,
                              void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                              void* stream);
 
+/* Head-range forms ("Sparse Transformer", llm-arch-kb, section 2, "How the
+ * two patterns are combined": the strided pattern on some heads and the fixed
+ * pattern on the rest, in equal proportion). They compute exactly what
+ * st_sparse_attn_fwd / st_sparse_attn_bwd compute, for heads h_begin ..
+ * h_begin + h_count - 1 of tensors with H heads, and leave every other head's
+ * rows of o, lse, dq, dk, dv untouched. Head indices stay global: a split
+ * layout still gives head h the set of its parity. Mixed heads are one call
+ * per layout on disjoint ranges; alternating patterns across layers is one
+ * layout per layer. Tensors, workspace size and errors are those of the
+ * full-range calls; ST_ERR_INVALID if the range is empty or leaves [0, H). */
+st_status st_sparse_attn_fwd_heads(const st_layout* layout, st_dtype dtype, int32_t B,
+                                   int32_t H, int32_t h_begin, int32_t h_count, int32_t T,
+                                   int32_t d, float scale, const void* q, const void* k,
+                                   const void* v, void* o, float* lse, void* stream);
+st_status st_sparse_attn_bwd_heads(const st_layout* layout, st_dtype dtype, int32_t B,
+                                   int32_t H, int32_t h_begin, int32_t h_count, int32_t T,
+                                   int32_t d, float scale, const void* q, const void* k,
+                                   const void* v, const void* o, const float* lse,
+                                   const void* dout, void* dq, void* dk, void* dv,
+                                   void* workspace, size_t ws_bytes, void* stream);
+
 /* Backward pass for callers that cannot allocate device memory. The paper
  * has no counterpart: this is a deployment convenience of this library.
  * Some callers cannot call cudaMalloc or keep a workspace between calls
