@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(PKG, "libsparse_transformer_attn.so")
 ST_OK, ST_ERR_INVALID, ST_ERR_UNSUPPORTED, ST_ERR_CUDA, ST_ERR_DEVICE_TIMEOUT, ST_ERR_WORKSPACE = range(6)
 ST_STRIDED, ST_FIXED, ST_DENSE_CAUSAL = 0, 1, 2
 ST_HEADS_SPLIT, ST_HEADS_MERGED = 0, 1
-ST_F32, ST_BF16 = 0, 1
+ST_F32, ST_BF16, ST_F16 = 0, 1, 2
 KINDS = {"strided": ST_STRIDED, "fixed": ST_FIXED, "dense": ST_DENSE_CAUSAL}
 MODES = {"split": ST_HEADS_SPLIT, "merged": ST_HEADS_MERGED}
 VIEWS = {0: "natural", 1: "summary", 2: "class"}
@@ -188,6 +188,8 @@ def _dtype_code(t):
         return ST_F32
     if t.dtype == torch.bfloat16:
         return ST_BF16
+    if t.dtype == torch.float16:
+        return ST_F16
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 

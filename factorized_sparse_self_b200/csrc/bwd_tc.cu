@@ -136,11 +136,12 @@ __device__ __forceinline__ void store_tile(const CUtensorMap* maps, int view, co
   }
 }
 
-// Eight fp32 values (bit patterns), times s, as four packed bf16 pairs.
+// Eight fp32 values (bit patterns), times s, as four packed 16-bit pairs.
+template <bool F16>
 __device__ __forceinline__ void round8(const uint32_t* v, float s, uint32_t w[4]) {
 #pragma unroll
   for (int x = 0; x < 4; ++x)
-    w[x] = pack_bf16(__uint_as_float(v[2 * x]) * s, __uint_as_float(v[2 * x + 1]) * s);
+    w[x] = pack2<F16>(__uint_as_float(v[2 * x]) * s, __uint_as_float(v[2 * x + 1]) * s);
 }
 
 // Live query columns [lo, hi) of a query tile for the key at natural
@@ -194,6 +195,7 @@ __device__ __forceinline__ Unit unit_of(const BwdItem* items, int u, int NH, con
   return x;
 }
 
+template <bool F16>  // 16-bit element type: fp16 if true, else bf16
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __restrict__ items,
               int n_units, int NH, const QEnt* __restrict__ qents, Heads hs,
@@ -387,9 +389,9 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     } else if (warp == 9) {
       // ---------------- MMA issuer ----------------
       if (lane == 0) {
-        const uint32_t idSS = idesc_bf16(128, 128, false, false);
-        const uint32_t idKM = idesc_bf16(128, 64, false, true);  // A K-major, B MN-major
-        const uint32_t idMM = idesc_bf16(128, 64, true, true);   // A MN-major, B MN-major
+        const uint32_t idSS = idesc_16(128, 128, false, false, F16);
+        const uint32_t idKM = idesc_16(128, 64, false, true, F16);  // A K-major, B MN-major
+        const uint32_t idMM = idesc_16(128, 64, true, true, F16);   // A MN-major, B MN-major
         const uint32_t ds_addr = smem_u32(S.dst);
         uint32_t k_addr = 0, v_addr = 0;
         bool ok = true;
@@ -569,7 +571,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t o4[4];
-          round8(dq + ch * 8, scale, o4);
+          round8<F16>(dq + ch * 8, scale, o4);
           st_shared_v4(st_addr + swz128(row, wg * 4 + ch), o4[0], o4[1], o4[2], o4[3]);
         }
       } else {
@@ -647,8 +649,8 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             float t0, t1, q0, q1;
             fadd2(t0, t1, dp[xk], dp[xk + 1], dv8[2 * x2], dv8[2 * x2 + 1]);
             fmul2(q0, q1, p0, p1, t0, t1);
-            pw[ch][x2] = pack_bf16(p0, p1);
-            dw[ch][x2] = pack_bf16(q0, q1);
+            pw[ch][x2] = pack2<F16>(p0, p1);
+            dw[ch][x2] = pack2<F16>(q0, q1);
           }
         }
         // the previous tile's dV, dK, dQ products are done with P^T, dS^T; at
@@ -699,7 +701,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t o4[4];
-          round8(r + ch * 8, sc, o4);
+          round8<F16>(r + ch * 8, sc, o4);
           st_shared_v4(dst + swz128(row, ch), o4[0], o4[1], o4[2], o4[3]);
         }
       } else {
@@ -725,23 +727,28 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
 
 }  // namespace
 
-cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, const float* lse,
-                   const void* dout, const float* D, float* dq_acc, float* dk_acc,
-                   float* dv_acc, void* dq, void* dk, void* dv, int* sched_counter) {
+namespace {
+
+template <bool F16>
+cudaError_t tc_bwd_t(const Call& c, const void* q, const void* k, const void* v,
+                     const float* lse, const void* dout, const float* D, float* dq_acc,
+                     float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv,
+                     int* sched_counter) {
   const st_layout* L = c.L;
   const int BH = c.B * c.H;
   if (L->dev.n_bwd_items == 0) return cudaSuccess;
   BwdMaps maps;
-  if (!make_view_maps(maps.q, q, false, L->geom, BH, c.d) ||
-      !make_view_maps(maps.k, k, false, L->geom, BH, c.d) ||
-      !make_view_maps(maps.v, v, false, L->geom, BH, c.d) ||
-      !make_view_maps(maps.dout, dout, false, L->geom, BH, c.d) ||
-      !make_view_maps(maps.dq, dq_acc, true, L->geom, BH, c.d) ||
-      !make_view_maps(maps.dk, dk_acc, true, L->geom, BH, c.d) ||
-      !make_view_maps(maps.dv, dv_acc, true, L->geom, BH, c.d) ||
-      !make_view_maps(maps.dqo, dq, false, L->geom, BH, c.d) ||
-      !make_view_maps(maps.dko, dk, false, L->geom, BH, c.d) ||
-      !make_view_maps(maps.dvo, dv, false, L->geom, BH, c.d))
+  const int el = F16 ? ELEM_F16 : ELEM_BF16;
+  if (!make_view_maps(maps.q, q, el, L->geom, BH, c.d) ||
+      !make_view_maps(maps.k, k, el, L->geom, BH, c.d) ||
+      !make_view_maps(maps.v, v, el, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dout, dout, el, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dq, dq_acc, ELEM_F32, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dk, dk_acc, ELEM_F32, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dv, dv_acc, ELEM_F32, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dqo, dq, el, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dko, dk, el, L->geom, BH, c.d) ||
+      !make_view_maps(maps.dvo, dv, el, L->geom, BH, c.d))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(SmemBwd);
   static_assert(sizeof(SmemBwd) <= 227 * 1024, "shared memory plan exceeds a CTA's 227 KB");
@@ -750,7 +757,7 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, c
   cudaGetDevice(&dev);
   cudaError_t err = cudaSuccess;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    err = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(bwd_tc_kernel<F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)smem);
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
@@ -767,7 +774,7 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, c
   if (units > 0x7fffffff) return cudaErrorInvalidValue;
   const int grid = (int)std::min<long long>(units, sms);
   record_begin(c);
-  bwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
+  bwd_tc_kernel<F16><<<grid, kThreads, smem, c.stream>>>(
       maps, L->geom, (const BwdItem*)L->dev.bwd_split[f], (int)units, NH,
       (const QEnt*)L->dev.q_ents, heads_of(c), c.scale, c.scale * kLog2e, lse, D,
       sched_counter, c.status,
@@ -775,6 +782,17 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, c
   err = cudaGetLastError();
   record_end(c);
   return err;
+}
+
+}  // namespace
+
+cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, const float* lse,
+                   const void* dout, const float* D, float* dq_acc, float* dk_acc,
+                   float* dv_acc, void* dq, void* dk, void* dv, int* sched_counter) {
+  return c.dtype == ST_F16 ? tc_bwd_t<true>(c, q, k, v, lse, dout, D, dq_acc, dk_acc, dv_acc,
+                                            dq, dk, dv, sched_counter)
+                           : tc_bwd_t<false>(c, q, k, v, lse, dout, D, dq_acc, dk_acc, dv_acc,
+                                             dq, dk, dv, sched_counter);
 }
 
 }  // namespace st

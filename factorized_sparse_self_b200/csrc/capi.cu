@@ -75,7 +75,7 @@ bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15
 st_status prepare(const st_layout* L, st_dtype dtype, int32_t B, int32_t H, int32_t h0, int32_t hn,
                   int32_t T, int32_t d, float scale, void* stream, Call& c) {
   if (!L || !L->on_device) return ST_ERR_INVALID;
-  if (dtype != ST_F32 && dtype != ST_BF16) return ST_ERR_INVALID;
+  if (dtype != ST_F32 && dtype != ST_BF16 && dtype != ST_F16) return ST_ERR_INVALID;
   if (B < 1 || H < 1 || d < 1 || T != L->geom.T) return ST_ERR_INVALID;
   if (h0 < 0 || hn < 1 || (int64_t)h0 + hn > H) return ST_ERR_INVALID;
   if ((int64_t)B * H > (1 << 30) || (int64_t)B * H * T * d > (int64_t)1 << 40) return ST_ERR_INVALID;
@@ -312,10 +312,10 @@ st_status st_sparse_attn_fwd_heads(const st_layout* L, st_dtype dtype, int32_t B
 st_status st_sparse_attn_bwd_workspace(const st_layout* L, st_dtype dtype, int32_t B, int32_t H,
                                        int32_t T, int32_t d, size_t* bytes) {
   if (!L || !bytes || B < 1 || H < 1 || d < 1 || T != L->geom.T) return ST_ERR_INVALID;
-  if (dtype != ST_F32 && dtype != ST_BF16) return ST_ERR_INVALID;
+  if (dtype != ST_F32 && dtype != ST_BF16 && dtype != ST_F16) return ST_ERR_INVALID;
   const size_t rows = (size_t)B * H * T;
   size_t b = round256(rows * sizeof(float));  // D
-  if (dtype == ST_BF16) b += 3 * round256(rows * (size_t)d * sizeof(float)) + 256;
+  if (dtype != ST_F32) b += 3 * round256(rows * (size_t)d * sizeof(float)) + 256;
   *bytes = b;
   return ST_OK;
 }
@@ -393,14 +393,14 @@ st_status st_last_device_status(void* stream) {
 }
 
 st_status st_layout_launches(const st_layout* L, st_dtype dtype, int32_t* fwd, int32_t* bwd) {
-  if (!L || (dtype != ST_F32 && dtype != ST_BF16)) return ST_ERR_INVALID;
+  if (!L || (dtype != ST_F32 && dtype != ST_BF16 && dtype != ST_F16)) return ST_ERR_INVALID;
   int32_t nf = 0;
   for (int p = 0; p < L->n_passes; ++p) nf += L->fwd_items[p].empty() ? 0 : 1;
   int32_t nb;
   if (dtype == ST_F32) {
     nb = 1 + (L->bwd_items.empty() ? 0 : 1) + nf;  // prologue, key-major kernel, dQ per pass
   } else {
-    nb = 2 + (L->bwd_items.empty() ? 0 : 1);       // prologue, main kernel, epilogue
+    nb = 2 + (L->bwd_items.empty() ? 0 : 1);       // prep, main kernel, finish
   }
   if (fwd) *fwd = nf;
   if (bwd) *bwd = nb;

@@ -146,10 +146,11 @@ __device__ __forceinline__ Unit unit_of(const FwdItem* items, int u, int NH, con
   return x;
 }
 
+template <bool F16>  // 16-bit element type: fp16 if true, else bf16
 __global__ void __launch_bounds__(kThreads, 2)
 fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __restrict__ items,
               int n_units, int NH, const KeyEnt* __restrict__ keys, Heads hs,
-              float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+              float scale_log2, uint16_t* __restrict__ out, float* __restrict__ lse,
               int* sched_slot, int* status, uint64_t wait_ns, int force_timeout) {
   extern __shared__ uint8_t smem_raw[];
   SmemFwd& S = *reinterpret_cast<SmemFwd*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -318,8 +319,8 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
   } else if (warp == 5) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t idS = idesc_bf16(128, 128, false, false);
-      const uint32_t idPV = idesc_bf16(128, 64, false, true);
+      const uint32_t idS = idesc_16(128, 128, false, false, F16);
+      const uint32_t idPV = idesc_16(128, 64, false, true, F16);
       bool ok = true;
       int gt = 0, n = 0;  // tiles and units of this CTA issued so far
       // S of global tile g from Q buffer qb and K ring stage g % NS.
@@ -489,7 +490,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int q2 = 0; q2 < 4; ++q2) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ws[q2]));
+            const float2 f = unpack2<F16>(ws[q2]);
             o[ch * 8 + 2 * q2] = fmaf(wp, f.x, wc * o[ch * 8 + 2 * q2]);
             o[ch * 8 + 2 * q2 + 1] = fmaf(wp, f.y, wc * o[ch * 8 + 2 * q2 + 1]);
           }
@@ -497,10 +498,10 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       }
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch)
-        dst[ch] = make_uint4(pack_bf16(o[ch * 8 + 0], o[ch * 8 + 1]),
-                             pack_bf16(o[ch * 8 + 2], o[ch * 8 + 3]),
-                             pack_bf16(o[ch * 8 + 4], o[ch * 8 + 5]),
-                             pack_bf16(o[ch * 8 + 6], o[ch * 8 + 7]));
+        dst[ch] = make_uint4(pack2<F16>(o[ch * 8 + 0], o[ch * 8 + 1]),
+                             pack2<F16>(o[ch * 8 + 2], o[ch * 8 + 3]),
+                             pack2<F16>(o[ch * 8 + 4], o[ch * 8 + 5]),
+                             pack2<F16>(o[ch * 8 + 6], o[ch * 8 + 7]));
       lse[(size_t)pe.bh * g.T + pe.i] = L;
     };
     auto epilogue = [&](const Pending& pe) {
@@ -590,7 +591,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
           const int j = (xk >> 1) & 3;
           fadd2(sa[j], sb[j], sa[j], sb[j], p0, p1);
-          pk[xk >> 1] = pack_bf16(p0, p1);
+          pk[xk >> 1] = pack2<F16>(p0, p1);
         }
         l_run = l_run * alpha + (((sa[0] + sb[0]) + (sa[1] + sb[1])) +
                                  ((sa[2] + sb[2]) + (sa[3] + sb[3])));
@@ -658,14 +659,18 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
 
 }  // namespace
 
-cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, void* o,
-                   float* lse, int force_timeout) {
+namespace {
+
+template <bool F16>
+cudaError_t tc_fwd_t(const Call& c, const void* q, const void* k, const void* v, void* o,
+                     float* lse, int force_timeout) {
   const st_layout* L = c.L;
   const int BH = c.B * c.H;
   FwdMaps maps;
-  if (!make_view_maps(maps.q, q, false, L->geom, BH, c.d) ||
-      !make_view_maps(maps.k, k, false, L->geom, BH, c.d) ||
-      !make_view_maps(maps.v, v, false, L->geom, BH, c.d))
+  const int el = F16 ? ELEM_F16 : ELEM_BF16;
+  if (!make_view_maps(maps.q, q, el, L->geom, BH, c.d) ||
+      !make_view_maps(maps.k, k, el, L->geom, BH, c.d) ||
+      !make_view_maps(maps.v, v, el, L->geom, BH, c.d))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(SmemFwd) + 1024;
   static bool attr_set[64] = {false};
@@ -673,7 +678,7 @@ cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, v
   cudaGetDevice(&dev);
   cudaError_t err = cudaSuccess;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    err = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(fwd_tc_kernel<F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)smem);
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
@@ -689,15 +694,23 @@ cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, v
     const long long units = (long long)n * NH;
     if (units > 0x7fffffff) return cudaErrorInvalidValue;
     const int grid = (int)std::min<long long>(units, 2LL * sms);
-    fwd_tc_kernel<<<grid, kThreads, smem, c.stream>>>(
+    fwd_tc_kernel<F16><<<grid, kThreads, smem, c.stream>>>(
         maps, L->geom, (const FwdItem*)L->dev.fwd_items[pass], (int)units, NH,
-        (const KeyEnt*)L->dev.key_ents, heads_of(c), scale_log2, (__nv_bfloat16*)o, lse,
+        (const KeyEnt*)L->dev.key_ents, heads_of(c), scale_log2, (uint16_t*)o, lse,
         slot, c.status, c.wait_ns, (force_timeout && pass == 0) ? 1 : 0);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
   record_end(c);
   return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, void* o,
+                   float* lse, int force_timeout) {
+  return c.dtype == ST_F16 ? tc_fwd_t<true>(c, q, k, v, o, lse, force_timeout)
+                           : tc_fwd_t<false>(c, q, k, v, o, lse, force_timeout);
 }
 
 }  // namespace st

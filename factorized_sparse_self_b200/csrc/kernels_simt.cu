@@ -296,20 +296,29 @@ RowSet row_set_of(const st_layout* L) {
 }
 
 // Grid (x, B*H); d = 64 bf16 rows of 128 bytes.
-__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
+// Dot product of eight 16-bit values (fp16 if F16, else bf16), in fp32.
+template <bool F16>
+__device__ __forceinline__ float dot8(const uint4& a, const uint4& b) {
   const uint32_t* x = reinterpret_cast<const uint32_t*>(&a);
   const uint32_t* y = reinterpret_cast<const uint32_t*>(&b);
   float s = 0.f;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const float2 u = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x[k]));
-    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y[k]));
+    float2 u, v;
+    if constexpr (F16) {
+      u = __half22float2(*reinterpret_cast<const __half2*>(&x[k]));
+      v = __half22float2(*reinterpret_cast<const __half2*>(&y[k]));
+    } else {
+      u = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x[k]));
+      v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y[k]));
+    }
     s = fmaf(u.x, v.x, s);
     s = fmaf(u.y, v.y, s);
   }
   return s;
 }
 
+template <bool F16>
 __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
                                 float* __restrict__ Dv,
                                 int T, Heads hs, RowSet rs, float4* __restrict__ dq_acc,
@@ -343,7 +352,7 @@ __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __rest
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        float sacc = dot8_bf16(a[u], b[u]);
+        float sacc = dot8<F16>(a[u], b[u]);
         sacc += __shfl_xor_sync(0xffffffffu, sacc, 4);
         sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
         sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
@@ -386,16 +395,26 @@ __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __rest
   }
 }
 
+template <bool F16>
+__device__ __forceinline__ uint32_t round2(float lo, float hi) {
+  if constexpr (F16) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+template <bool F16>
 __device__ __forceinline__ uint4 round8f(const float4& a, const float4& b, float s) {
-  __nv_bfloat162 w[4] = {__floats2bfloat162_rn(a.x * s, a.y * s),
-                         __floats2bfloat162_rn(a.z * s, a.w * s),
-                         __floats2bfloat162_rn(b.x * s, b.y * s),
-                         __floats2bfloat162_rn(b.z * s, b.w * s)};
-  return *reinterpret_cast<uint4*>(w);
+  return make_uint4(round2<F16>(a.x * s, a.y * s), round2<F16>(a.z * s, a.w * s),
+                    round2<F16>(b.x * s, b.y * s), round2<F16>(b.z * s, b.w * s));
 }
 
 // Rounds the accumulated rows: eight elements (two float4 in, 16 bytes out)
 // per thread and step.
+template <bool F16>
 __global__ void bwd_finish_kernel(const float4* __restrict__ dq_acc,
                                   const float4* __restrict__ dk_acc,
                                   const float4* __restrict__ dv_acc, int T, Heads hs,
@@ -411,7 +430,7 @@ __global__ void bwd_finish_kernel(const float4* __restrict__ dq_acc,
     const int32_t* rows = rows_of(rs, hc, ROWS_Q_ACC, nr);
     for (int64_t x = tid; x < (int64_t)nr * 8; x += stride) {
       const size_t e = (rb + rows[x >> 3]) * 8 + (x & 7);
-      dq[e] = round8f(__ldg(dq_acc + 2 * e), __ldg(dq_acc + 2 * e + 1), scale);
+      dq[e] = round8f<F16>(__ldg(dq_acc + 2 * e), __ldg(dq_acc + 2 * e + 1), scale);
     }
   }
   {
@@ -419,8 +438,8 @@ __global__ void bwd_finish_kernel(const float4* __restrict__ dq_acc,
     const int32_t* rows = rows_of(rs, hc, ROWS_K_ACC, nr);
     for (int64_t x = tid; x < (int64_t)nr * 8; x += stride) {
       const size_t e = (rb + rows[x >> 3]) * 8 + (x & 7);
-      dk[e] = round8f(__ldg(dk_acc + 2 * e), __ldg(dk_acc + 2 * e + 1), scale);
-      dv[e] = round8f(__ldg(dv_acc + 2 * e), __ldg(dv_acc + 2 * e + 1), 1.f);
+      dk[e] = round8f<F16>(__ldg(dk_acc + 2 * e), __ldg(dk_acc + 2 * e + 1), scale);
+      dv[e] = round8f<F16>(__ldg(dv_acc + 2 * e), __ldg(dv_acc + 2 * e + 1), 1.f);
     }
   }
 }
@@ -523,13 +542,9 @@ cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* 
   size_t rows = (size_t)c.B * c.H * c.L->geom.T;
   int threads = 256;
   int blocks = grid_cap(rows * 32 > acc_elems / 4 ? rows * 32 : acc_elems / 4, threads);
-  if (c.dtype == ST_F32)
-    prologue_kernel<float><<<blocks, threads, 0, c.stream>>>(
-        (const float*)o, (const float*)dout, Dv, rows, c.d, (float4*)acc, acc_elems / 4);
-  else
-    prologue_kernel<__nv_bfloat16><<<blocks, threads, 0, c.stream>>>(
-        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, Dv, rows, c.d, (float4*)acc,
-        acc_elems / 4);
+  if (c.dtype != ST_F32) return cudaErrorInvalidValue;  // 16-bit calls use bwd_prep
+  prologue_kernel<float><<<blocks, threads, 0, c.stream>>>(
+      (const float*)o, (const float*)dout, Dv, rows, c.d, (float4*)acc, acc_elems / 4);
   return cudaGetLastError();
 }
 
@@ -539,7 +554,8 @@ cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* Dv, 
   const int T = c.L->geom.T;
   const int bx = std::max(1, std::min(64, (T + 127) / 128));
   dim3 grid(bx, c.B * c.hn);
-  bwd_prep_kernel<<<grid, 256, 0, c.stream>>>(
+  auto kern = (c.dtype == ST_F16) ? bwd_prep_kernel<true> : bwd_prep_kernel<false>;
+  kern<<<grid, 256, 0, c.stream>>>(
       (const uint4*)o, (const uint4*)dout, Dv, T, heads_of(c),
       row_set_of(c.L), (float4*)dq_acc, (float4*)dk_acc, (float4*)dv_acc, (uint4*)dq, (uint4*)dk,
       (uint4*)dv, sched_counter);
@@ -555,7 +571,8 @@ cudaError_t bwd_finish(const Call& c, const float* dq_acc, const float* dk_acc,
   if (most == 0) return cudaSuccess;  // every row was written directly
   const int bx = std::max(1, std::min(64, (most + 31) / 32));
   dim3 grid(bx, c.B * c.hn);
-  bwd_finish_kernel<<<grid, 256, 0, c.stream>>>(
+  auto kern = (c.dtype == ST_F16) ? bwd_finish_kernel<true> : bwd_finish_kernel<false>;
+  kern<<<grid, 256, 0, c.stream>>>(
       (const float4*)dq_acc, (const float4*)dk_acc, (const float4*)dv_acc, L->geom.T,
       heads_of(c), row_set_of(L), c.scale, (uint4*)dq, (uint4*)dk, (uint4*)dv);
   return cudaGetLastError();

@@ -94,11 +94,18 @@ inline int heads_per_class(const Call& c) {
   return c.B * most;
 }
 
+// Element types of tensor maps.
+enum Elem : int { ELEM_BF16 = 0, ELEM_F16 = 1, ELEM_F32 = 2 };
+
 // Encodes the natural (3-D), summary and residue-class (4-D) TMA views of a
-// [B*H, T, d] tensor: bf16 with 64-element boxes, or fp32 with 32-element
-// boxes; 128-byte swizzle; 128-row boxes. Views the layout lacks get a copy
-// of the natural map (never used). Returns false if the driver rejects one.
-bool make_view_maps(CUtensorMap out[3], const void* base, bool is_f32, const Geom& g, int BH,
+// [B*H, T, d] tensor: 16-bit elements with 64-element boxes, or fp32 with
+// 32-element boxes; 128-byte swizzle; 128-row boxes. Views the layout lacks
+// get a copy of the natural map (never used). Returns false if the driver
+// rejects one.
+bool make_view_maps(CUtensorMap out[3], const void* base, int elem, const Geom& g, int BH,
                     int d);
+
+// Element type of a call's 16-bit tensors.
+inline int elem16(const Call& c) { return c.dtype == ST_F16 ? ELEM_F16 : ELEM_BF16; }
 
 }  // namespace st

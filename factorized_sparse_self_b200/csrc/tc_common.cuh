@@ -356,13 +356,17 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
   return d;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A and B and an fp32 D:
-// D format bits 4-5 (1 = f32), A format bits 7-9 and B format bits 10-12
-// (1 = bf16), A / B major bits 15 / 16 (1 = MN-major), N >> 3 in bits 17-22,
-// M >> 4 in bits 24-28.
+// Instruction descriptor of kind::f16 with 16-bit A and B (both fp16, or
+// both bf16) and an fp32 D: D format bits 4-5 (1 = f32), A format bits 7-9
+// and B format bits 10-12 (0 = f16, 1 = bf16), A / B major bits 15 / 16
+// (1 = MN-major), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_16(int M, int N, bool a_mn, bool b_mn, bool f16) {
+  return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) |
+         ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
-         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+  return idesc_16(M, N, a_mn, b_mn, false);
 }
 
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128B-swizzled
@@ -374,6 +378,25 @@ __device__ __forceinline__ uint32_t swz128(int row, int chunk) {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Two floats rounded to the 16-bit element type (fp16 if F16, else bf16),
+// low half first; and back.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (F16) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    return pack_bf16(lo, hi);
+  }
+}
+template <bool F16>
+__device__ __forceinline__ float2 unpack2(uint32_t u) {
+  if constexpr (F16)
+    return __half22float2(*reinterpret_cast<const __half2*>(&u));
+  else
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,

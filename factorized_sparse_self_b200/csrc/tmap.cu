@@ -31,12 +31,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool encode_views(CUtensorMap out[3], const void* base, bool is_f32, const Geom& g, int BH,
-                  int d) {
+bool encode_views(CUtensorMap out[3], const void* base, int elem, const Geom& g, int BH, int d) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  const CUtensorMapDataType dt =
-      is_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const bool is_f32 = (elem == ELEM_F32);
+  const CUtensorMapDataType dt = is_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : elem == ELEM_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const cuuint64_t es = is_f32 ? 4 : 2;
   const cuuint32_t inner = is_f32 ? 32 : 64;
   const cuuint64_t row = (cuuint64_t)d * es;
@@ -74,7 +75,7 @@ bool encode_views(CUtensorMap out[3], const void* base, bool is_f32, const Geom&
 
 struct Key {
   const void* base;
-  int is_f32, T, l, c, P, nsum, BH, d;
+  int elem, T, l, c, P, nsum, BH, d;
   bool operator==(const Key& o) const { return std::memcmp(this, &o, sizeof(Key)) == 0; }
 };
 
@@ -92,12 +93,12 @@ std::mutex g_cache_mu;
 
 }  // namespace
 
-bool make_view_maps(CUtensorMap out[3], const void* base, bool is_f32, const Geom& g, int BH,
+bool make_view_maps(CUtensorMap out[3], const void* base, int elem, const Geom& g, int BH,
                     int d) {
   Key key;
   std::memset(&key, 0, sizeof(key));
   key.base = base;
-  key.is_f32 = is_f32 ? 1 : 0;
+  key.elem = elem;
   key.T = g.T;
   key.l = g.l;
   key.c = g.c;
@@ -118,7 +119,7 @@ bool make_view_maps(CUtensorMap out[3], const void* base, bool is_f32, const Geo
                        (!g_cache[e].valid || g_cache[e].stamp < g_cache[victim].stamp)))
       victim = e;
   }
-  if (!encode_views(out, base, is_f32, g, BH, d)) return false;
+  if (!encode_views(out, base, elem, g, BH, d)) return false;
   g_cache[victim].key = key;
   std::memcpy(g_cache[victim].maps, out, sizeof(g_cache[victim].maps));
   g_cache[victim].stamp = ++g_clock;

@@ -29,7 +29,7 @@ def main():
     ap.add_argument("--d", type=int, default=64)
     ap.add_argument("--l", type=int, default=128)
     ap.add_argument("--c", type=int, default=8)
-    ap.add_argument("--dtype", default="bf16", choices=["bf16", "f32"])
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16", "f32"])
     ap.add_argument("--iters", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--fwd-only", action="store_true")
@@ -52,7 +52,7 @@ def main():
     o = torch.empty_like(q)
     lse = torch.empty((a.B, a.H, a.T), dtype=torch.float32, device="cuda")
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    code = st.ST_BF16 if a.dtype == "bf16" else st.ST_F32
+    code = {"bf16": st.ST_BF16, "f16": st.ST_F16, "f32": st.ST_F32}[a.dtype]
     ws = torch.empty(st.st_sparse_attn_bwd_workspace(L, code, a.B, a.H, a.T, a.d),
                      dtype=torch.uint8, device="cuda")
 

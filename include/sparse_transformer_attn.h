@@ -35,8 +35,8 @@
  *  - Errors are returned as st_status; nothing is thrown across the ABI.
  *    Invalid arguments return ST_ERR_INVALID before any launch; shapes the
  *    kernels do not implement return ST_ERR_UNSUPPORTED before any launch.
- *  - Supported shapes: bf16 with d = 64 (tensor-core path), float32 with
- *    d = 32 or 64 (exact fp32 path). T must be a multiple of 128; l must
+ *  - Supported shapes: bf16 or fp16 with d = 64 (tensor-core path), float32
+ *    with d = 32 or 64 (exact fp32 path). T must be a multiple of 128; l must
  *    divide T or be >= T; for the fixed pattern with l < T, c must divide 128
  *    and satisfy 1 <= c <= l.
  */
@@ -61,7 +61,10 @@ typedef enum {
 
 typedef enum { ST_STRIDED = 0, ST_FIXED = 1, ST_DENSE_CAUSAL = 2 } st_pattern_kind;
 typedef enum { ST_HEADS_SPLIT = 0, ST_HEADS_MERGED = 1 } st_head_mode;
-typedef enum { ST_F32 = 0, ST_BF16 = 1 } st_dtype;
+/* ST_F16: IEEE half precision, for the 16-bit mixed precision of the
+ * milestone page ("The idea"); it runs the same tensor-core kernels as bf16, with
+ * P and dS rounded to fp16 instead of bf16 and fp32 accumulation. */
+typedef enum { ST_F32 = 0, ST_BF16 = 1, ST_F16 = 2 } st_dtype;
 
 /* Pattern of one attention layer. l is the stride / block length
  * ("Sparse Transformer", llm-arch-kb, section 2: l ~ sqrt(T)); c is the number

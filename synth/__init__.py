@@ -28,7 +28,7 @@ class Workload:
     d: int
     l: int
     c: int
-    dtype: str         # "f32" | "bf16"
+    dtype: str         # "f32" | "bf16" | "f16"
     std: float         # standard deviation of Q, K, V
     backward: bool = True
     note: str = field(default="", compare=False)
@@ -55,7 +55,7 @@ ORDER = list(WORKLOADS)
 
 
 def torch_dtype(name: str) -> torch.dtype:
-    return {"f32": torch.float32, "bf16": torch.bfloat16}[name]
+    return {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[name]
 
 
 def draw(B, H, T, d, dtype="bf16", std=1.0, seed=0, dout_std=1.0):

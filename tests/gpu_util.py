@@ -9,8 +9,12 @@ import factorized_sparse_self_b200 as st
 import synth
 
 # Tolerances: fp32 max-abs 1e-4; bf16 max-abs 2e-2 and relative L2 1e-2 per
-# output tensor, the oracle being fed the bf16-rounded inputs.
-TOL = {"f32": {"abs": 1e-4, "rel": None}, "bf16": {"abs": 2e-2, "rel": 1e-2}}
+# output tensor, the oracle being fed the bf16-rounded inputs. fp16 runs the
+# same kernels with every 16-bit rounding (P, dS and the outputs) eight times
+# finer (unit roundoff 2^-11 against 2^-8), so its bounds are the bf16 ones
+# divided by 5 (a margin of 8/5 over the scaled bf16 bounds).
+TOL = {"f32": {"abs": 1e-4, "rel": None}, "bf16": {"abs": 2e-2, "rel": 1e-2},
+       "f16": {"abs": 4e-3, "rel": 2e-3}}
 
 
 def rel_l2(x, y):
