@@ -62,6 +62,15 @@ struct BwdMaps {
   CUtensorMap dqo[3], dko[3], dvo[3];     // bf16 outputs (direct tiles)
 };
 
+// A published work unit: its index (n_units: no more work), head, item and
+// query entries, so that no consuming role reads the schedule from global
+// memory at a unit boundary.
+struct SchedSlot {
+  int u, bh;
+  BwdItem it;
+  QEnt q[kBwdChunk];
+};
+
 struct SmemBwd {
   uint8_t k[2][kTileBytes];
   uint8_t v[2][kTileBytes];
@@ -69,14 +78,14 @@ struct SmemBwd {
   uint8_t dout[NS][kTileBytes];
   uint8_t dst[2 * kTileBytes];   // dS^T (keys x queries), two 64-query K-blocks
   uint8_t stage[2 * kTileBytes]; // dQ tile: fp32 in two 32-column halves, or bf16
-  uint8_t kvst[2 * kTileBytes];  // dK tile at the end of a unit (dV goes through dst)
+  uint8_t kvst[2 * kTileBytes];  // end of a unit: dK (fp32), or dK and dV (bf16 / fp16)
   float l2[NS][kTile];           // -LSE_i * log2(e) of the stage's query rows
   float dd[NS][kTile];           // -D_i
   uint64_t kv_full[2], kv_done[2], full[NS], empty[NS];
   uint64_t s_full, dp_full, sdp_free, ds_ready, pds_free, dq_full, dq_free, stg_full, stg_free;
-  uint64_t acc_full, acc_free, out_full, kvstg_free, fin;
+  uint64_t acc_full, acc_free, out_full, dst_free, kvst_free, fin;
   uint64_t sched_full[kSched], sched_empty[kSched];
-  int sched[kSched];             // work unit of each slot (n_units: no more work)
+  SchedSlot slot[kSched];        // published units
   uint32_t tmem_base;
   int abort;
 };
@@ -235,7 +244,8 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     mbar_init(&S.acc_full, 1);
     mbar_init(&S.acc_free, 256);
     mbar_init(&S.out_full, 256);
-    mbar_init(&S.kvstg_free, 1);
+    mbar_init(&S.dst_free, 1);
+    mbar_init(&S.kvst_free, 1);
     mbar_init(&S.fin, 1);
     for (int k = 0; k < kSched; ++k) {
       mbar_init(&S.sched_full[k], 1);
@@ -255,15 +265,14 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     *abort = 1;
     set_status(status, ST_ERR_DEVICE_TIMEOUT);
   };
-  // Next published unit for a consuming role; `arrive` releases the slot
-  // (one arrival per consuming warp).
+  // Next published unit for a consuming role: its slot k. A role releases
+  // the slot (one arrival per consuming warp) once it has finished the unit.
   int sk = 0;
-  auto next_unit = [&](int& u, bool arrive) -> bool {
-    const int k = sk % kSched;
+  auto next_unit = [&](int& u, int& k) -> bool {
+    k = sk % kSched;
     const bool w = mbar_wait(&S.sched_full[k], (sk / kSched) & 1, wait_ns, abort);
     if (!w) return false;
-    u = *reinterpret_cast<volatile int*>(&S.sched[k]);
-    if (arrive) mbar_arrive(&S.sched_empty[k]);
+    u = *reinterpret_cast<volatile int*>(&S.slot[k].u);
     ++sk;
     return true;
   };
@@ -292,10 +301,18 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         const int k = pub % kSched;
         const bool w = mbar_wait(&S.sched_empty[k], ((pub / kSched) & 1) ^ 1, wait_ns, abort);
         if (!__all_sync(0xffffffffu, w)) return false;
-        if (lane == 0) {
-          S.sched[k] = u;
-          mbar_arrive(&S.sched_full[k]);
+        SchedSlot& sl = S.slot[k];
+        if (u < n_units) {
+          const Unit x = unit_of(items, u, NH, hs);
+          if (lane < x.it.qend - x.it.qbeg) sl.q[lane] = qents[x.it.qbeg + lane];
+          if (lane == 0) {
+            sl.bh = x.bh;
+            sl.it = x.it;
+          }
         }
+        if (lane == 0) sl.u = u;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.sched_full[k]);
         ++pub;
         return true;
       };
@@ -414,14 +431,13 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           return true;
         };
         for (;;) {
-          int u = 0;
-          if (!next_unit(u, true)) {
+          int u = 0, sl = 0;
+          if (!next_unit(u, sl)) {
             ok = false;
             break;
           }
           if (u >= n_units) break;
-          const Unit x = unit_of(items, u, NH, hs);
-          const int cnt = x.it.qend - x.it.qbeg;
+          const int cnt = S.slot[sl].it.qend - S.slot[sl].it.qbeg;
           const int kb = n & 1;
           k_addr = smem_u32(S.k[kb]);
           v_addr = smem_u32(S.v[kb]);
@@ -474,6 +490,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             mma_commit(&S.pds_free);
           }
           if (!ok) break;
+          mbar_arrive(&S.sched_empty[sl]);
           mma_commit(&S.kv_done[n & 1]);
           mma_commit(&S.acc_full);
           ++n;
@@ -500,20 +517,22 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           return true;
         };
         for (;;) {
-          int u = 0;
-          if (!next_unit(u, true)) {
+          int u = 0, sl = 0;
+          if (!next_unit(u, sl)) {
             ok = false;
             break;
           }
           if (u >= n_units) break;
-          const Unit x = unit_of(items, u, NH, hs);
+          Unit x;
+          x.it = S.slot[sl].it;
+          x.bh = S.slot[sl].bh;
           const int cnt = x.it.qend - x.it.qbeg;
           for (int e = 0; ok && e < cnt; ++e, ++gt) {
             if (gt > 0 && !reduce_dq(gt - 1)) {
               ok = false;
               break;
             }
-            const QEnt qe = qents[x.it.qbeg + e];
+            const QEnt qe = S.slot[sl].q[e];
             pv = x.it.qview;
             ptile = qe.qtile;
             pdirect = qe.q_direct;
@@ -524,16 +543,22 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             ok = false;
             break;
           }
-          if (x.it.kv_direct) {
+          if (x.it.kv_direct) {  // both 16-bit tiles in kvst; dst was not used
+            mbar_arrive(&S.dst_free);
             store_tile(maps.dko, x.it.kview, g, x.it.ktile, x.bh, S.kvst);
-            store_tile(maps.dvo, x.it.kview, g, x.it.ktile, x.bh, S.dst);
-          } else {
-            reduce_tile(maps.dk, x.it.kview, g, x.it.ktile, x.bh, S.kvst);
+            store_tile(maps.dvo, x.it.kview, g, x.it.ktile, x.bh, S.kvst + kTileBytes);
+            bulk_commit();
+          } else {  // dV (in dst) first: the next unit's first dS^T waits for it
             reduce_tile(maps.dv, x.it.kview, g, x.it.ktile, x.bh, S.dst);
+            bulk_commit();
+            reduce_tile(maps.dk, x.it.kview, g, x.it.ktile, x.bh, S.kvst);
+            bulk_commit();
+            bulk_wait_read_le1();
+            mbar_arrive(&S.dst_free);
           }
-          bulk_commit();
           bulk_wait_read_all();
-          mbar_arrive(&S.kvstg_free);
+          mbar_arrive(&S.kvst_free);
+          mbar_arrive(&S.sched_empty[sl]);
           ++n;
         }
         if (ok && gt > 0 && !reduce_dq(gt - 1)) ok = false;
@@ -586,22 +611,22 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     };
 
     for (;;) {
-      int u = 0;
-      const bool got = next_unit(u, false);
-      __syncwarp();
-      if (lane == 0 && got) mbar_arrive(&S.sched_empty[(sk - 1) % kSched]);
+      int u = 0, sl = 0;
+      const bool got = next_unit(u, sl);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
       if (u >= n_units) break;
-      const Unit x = unit_of(items, u, NH, hs);
+      Unit x;
+      x.it = S.slot[sl].it;
+      x.bh = S.slot[sl].bh;
       const BwdItem& it = x.it;
       const int cnt = it.qend - it.qbeg;
       const int j = view_pos(g, it.kview, it.ktile, row);
       for (int e = 0; e < cnt; ++e, ++gt) {
         const int s = gt % NS;
-        const QEnt qe = qents[it.qbeg + e];
+        const QEnt qe = S.slot[sl].q[e];
         bool w = mbar_wait(&S.s_full, gt & 1, wait_ns, abort);
         w = w && mbar_wait(&S.dp_full, gt & 1, wait_ns, abort);
         w = w && mbar_wait(&S.full[s], (gt / NS) & 1, wait_ns, abort);
@@ -655,10 +680,10 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         }
         // the previous tile's dV, dK, dQ products are done with P^T, dS^T; at
         // the start of a unit the writer has also read the previous unit's
-        // dK, dV staging (dV sits in the dS^T buffer)
+        // fp32 dV staging, which sits in the dS^T buffer
         w = true;
         if (gt > 0) w = mbar_wait(&S.pds_free, (gt - 1) & 1, wait_ns, abort);
-        if (e == 0 && n > 0) w = w && mbar_wait(&S.kvstg_free, (n - 1) & 1, wait_ns, abort);
+        if (e == 0 && n > 0) w = w && mbar_wait(&S.dst_free, (n - 1) & 1, wait_ns, abort);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
@@ -693,9 +718,19 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&S.acc_free);
-      // stage for the writer warp: dK in its own buffer, dV in the dS^T buffer
-      // (free: every product of the unit has completed)
-      const uint32_t dst = wg ? ds_addr : smem_u32(S.kvst);
+      // stage for the writer warp: 16-bit dK and dV both in kvst; fp32 dK in
+      // kvst and fp32 dV in the dS^T buffer (free: every product of the unit
+      // has completed). kvst must have been read for the previous unit.
+      if (n > 0) {
+        w = mbar_wait(&S.kvst_free, (n - 1) & 1, wait_ns, abort);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+      }
+      const uint32_t kv_addr = smem_u32(S.kvst);
+      const uint32_t dst =
+          it.kv_direct ? kv_addr + (wg ? kTileBytes : 0) : (wg ? ds_addr : kv_addr);
       if (it.kv_direct) {
         const float sc = wg ? 1.f : scale;  // dK carries the softmax scale, dV none
 #pragma unroll
@@ -715,6 +750,8 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       }
       fence_async_smem();
       mbar_arrive(&S.out_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.sched_empty[sl]);  // this warp is done with the slot
       ++n;
     }
     if (ok && gt > 0 && !drain_dq(gt - 1, pend_direct)) ok = false;
