@@ -46,7 +46,7 @@ namespace {
 using namespace tc;
 
 constexpr int NS = 2;
-constexpr int kSched = 4;                   // published work units in flight
+constexpr int kSched = 6;                   // published work units in flight
 constexpr int kTileBytes = kTile * 64 * 2;  // 128 x 64 bf16 = 16 KB
 constexpr int kThreads = 384;
 constexpr uint32_t kRegsCompute = 200, kRegsIssue = 104;  // launch: 168 per thread
@@ -115,20 +115,20 @@ __device__ __forceinline__ void prefetch_tile(const CUtensorMap* maps, int view,
   }
 }
 
-// Reduce-adds a 128-row fp32 tile, staged as two 32-column halves.
-__device__ __forceinline__ void reduce_tile(const CUtensorMap* maps, int view, const Geom& g,
-                                            int tile, int bh, const uint8_t* src) {
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint8_t* s = src + h * kTileBytes;
-    if (view == VIEW_NAT) {
-      tma_reduce_add_3d(&maps[VIEW_NAT], s, h * 32, tile * kTile, bh);
-    } else if (view == VIEW_SUM) {
-      tma_reduce_add_4d(&maps[VIEW_SUM], s, h * 32, g.l - g.c, tile * (kTile / g.c), bh);
-    } else {
-      int r = tile / g.ptiles, pb = tile - r * g.ptiles;
-      tma_reduce_add_4d(&maps[VIEW_CLS], s, h * 32, r, pb * kTile, bh);
-    }
+// Reduce-adds one 32-column half h of a 128-row fp32 tile staged as two
+// halves. (TMA copies issued by one thread are processed one after another,
+// copies of different threads in parallel: the two halves go out from two
+// lanes.)
+__device__ __forceinline__ void reduce_half(const CUtensorMap* maps, int view, const Geom& g,
+                                            int tile, int bh, const uint8_t* src, int h) {
+  const uint8_t* s = src + h * kTileBytes;
+  if (view == VIEW_NAT) {
+    tma_reduce_add_3d(&maps[VIEW_NAT], s, h * 32, tile * kTile, bh);
+  } else if (view == VIEW_SUM) {
+    tma_reduce_add_4d(&maps[VIEW_SUM], s, h * 32, g.l - g.c, tile * (kTile / g.c), bh);
+  } else {
+    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+    tma_reduce_add_4d(&maps[VIEW_CLS], s, h * 32, r, pb * kTile, bh);
   }
 }
 
@@ -343,15 +343,15 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           }
           const bool w = mbar_wait(&S.empty[s], ((gt / NS) & 1) ^ 1, wait_ns, abort);
           if (!__all_sync(0xffffffffu, w)) return false;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&S.full[s], 2 * kTileBytes);
-            load_tile(S.q[s], maps.q, x.it.qview, g, qe.qtile, x.bh, &S.full[s]);
-            load_tile(S.dout[s], maps.dout, x.it.qview, g, qe.qtile, x.bh, &S.full[s]);
-            if (pf >= 0) {  // two tiles ahead of the ring: into L2 now
-              prefetch_tile(maps.q, x.it.qview, g, pf, x.bh);
-              prefetch_tile(maps.dout, x.it.qview, g, pf, x.bh);
-            }
-          }
+          if (lane == 0) mbar_arrive_expect_tx(&S.full[s], 2 * kTileBytes);
+          __syncwarp();
+          // Q from lane 0, dO from lane 1; the L2 prefetches of the tile two
+          // ahead from lanes 2, 3 (each thread's copies run one at a time)
+          if (lane < 2)
+            load_tile(lane ? S.dout[s] : S.q[s], lane ? maps.dout : maps.q, x.it.qview, g,
+                      qe.qtile, x.bh, &S.full[s]);
+          else if (lane < 4 && pf >= 0)
+            prefetch_tile(lane == 3 ? maps.dout : maps.q, x.it.qview, g, pf, x.bh);
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             const int row = lane + 32 * t;
@@ -372,11 +372,11 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           const int kb = m & 1;
           const bool w = mbar_wait(&S.kv_done[kb], ((m >> 1) & 1) ^ 1, wait_ns, abort);
           if (!__all_sync(0xffffffffu, w)) return false;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&S.kv_full[kb], 2 * kTileBytes);
-            load_tile(S.k[kb], maps.k, y.it.kview, g, y.it.ktile, y.bh, &S.kv_full[kb]);
-            load_tile(S.v[kb], maps.v, y.it.kview, g, y.it.ktile, y.bh, &S.kv_full[kb]);
-          }
+          if (lane == 0) mbar_arrive_expect_tx(&S.kv_full[kb], 2 * kTileBytes);
+          __syncwarp();
+          if (lane < 2)  // K from lane 0, V from lane 1
+            load_tile(lane ? S.v[kb] : S.k[kb], lane ? maps.v : maps.k, y.it.kview, g,
+                      y.it.ktile, y.bh, &S.kv_full[kb]);
           kv_last = m;
           return true;
         };
@@ -500,71 +500,84 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         mbar_wait(&S.fin, 0, wait_ns, abort);
       }
     } else if (warp == 10) {
-      // ---------------- reducer: TMA reduce-adds of the staged fp32 tiles ----------------
-      if (lane == 0) {
-        bool ok = true;
-        int gt = 0, n = 0;
-        int pv = 0, ptile = 0, pbh = 0, pdirect = 0;  // query tile of tile gt - 1
-        auto reduce_dq = [&](int t) -> bool {
-          if (!mbar_wait(&S.stg_full, t & 1, wait_ns, abort)) return false;
-          if (pdirect)
-            store_tile(maps.dqo, pv, g, ptile, pbh, S.stage);
-          else
-            reduce_tile(maps.dq, pv, g, ptile, pbh, S.stage);
+      // ---------------- writer: TMA stores / reduce-adds of the staged tiles ----------------
+      // Every copy goes out from a lane of its own, so that they run in parallel.
+      bool ok = true;
+      int gt = 0, n = 0;
+      int pv = 0, ptile = 0, pbh = 0, pdirect = 0;  // query tile of tile gt - 1
+      auto reduce_dq = [&](int t) -> bool {
+        const bool w = mbar_wait(&S.stg_full, t & 1, wait_ns, abort);
+        if (!__all_sync(0xffffffffu, w)) return false;
+        if (pdirect) {
+          if (lane == 0) store_tile(maps.dqo, pv, g, ptile, pbh, S.stage);
+        } else if (lane < 2) {
+          reduce_half(maps.dq, pv, g, ptile, pbh, S.stage, lane);
+        }
+        if (lane < 2) {
           bulk_commit();
           bulk_wait_read_all();
-          mbar_arrive(&S.stg_free);
-          return true;
-        };
-        for (;;) {
-          int u = 0, sl = 0;
-          if (!next_unit(u, sl)) {
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.stg_free);
+        return true;
+      };
+      for (;;) {
+        int u = 0, sl = 0;
+        const bool got = next_unit(u, sl);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        if (u >= n_units) break;
+        Unit x;
+        x.it = S.slot[sl].it;
+        x.bh = S.slot[sl].bh;
+        const int cnt = x.it.qend - x.it.qbeg;
+        for (int e = 0; ok && e < cnt; ++e, ++gt) {
+          if (gt > 0 && !reduce_dq(gt - 1)) {
             ok = false;
             break;
           }
-          if (u >= n_units) break;
-          Unit x;
-          x.it = S.slot[sl].it;
-          x.bh = S.slot[sl].bh;
-          const int cnt = x.it.qend - x.it.qbeg;
-          for (int e = 0; ok && e < cnt; ++e, ++gt) {
-            if (gt > 0 && !reduce_dq(gt - 1)) {
-              ok = false;
-              break;
-            }
-            const QEnt qe = S.slot[sl].q[e];
-            pv = x.it.qview;
-            ptile = qe.qtile;
-            pdirect = qe.q_direct;
-            pbh = x.bh;
-          }
-          if (!ok) break;
-          if (!mbar_wait(&S.out_full, n & 1, wait_ns, abort)) {
-            ok = false;
-            break;
-          }
-          if (x.it.kv_direct) {  // both 16-bit tiles in kvst; dst was not used
-            mbar_arrive(&S.dst_free);
-            store_tile(maps.dko, x.it.kview, g, x.it.ktile, x.bh, S.kvst);
-            store_tile(maps.dvo, x.it.kview, g, x.it.ktile, x.bh, S.kvst + kTileBytes);
+          const QEnt qe = S.slot[sl].q[e];
+          pv = x.it.qview;
+          ptile = qe.qtile;
+          pdirect = qe.q_direct;
+          pbh = x.bh;
+        }
+        if (!ok) break;
+        const bool w = mbar_wait(&S.out_full, n & 1, wait_ns, abort);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        if (x.it.kv_direct) {  // both 16-bit tiles in kvst; dst was not used
+          if (lane == 0) mbar_arrive(&S.dst_free);
+          if (lane < 2) {
+            store_tile(lane ? maps.dvo : maps.dko, x.it.kview, g, x.it.ktile, x.bh,
+                       S.kvst + lane * kTileBytes);
             bulk_commit();
-          } else {  // dV (in dst) first: the next unit's first dS^T waits for it
-            reduce_tile(maps.dv, x.it.kview, g, x.it.ktile, x.bh, S.dst);
-            bulk_commit();
-            reduce_tile(maps.dk, x.it.kview, g, x.it.ktile, x.bh, S.kvst);
-            bulk_commit();
-            bulk_wait_read_le1();
-            mbar_arrive(&S.dst_free);
           }
-          bulk_wait_read_all();
+        } else {  // lanes 0, 1: dV halves (in dst), read first; lanes 2, 3: dK halves
+          if (lane < 4) {
+            reduce_half(lane < 2 ? maps.dv : maps.dk, x.it.kview, g, x.it.ktile, x.bh,
+                        lane < 2 ? S.dst : S.kvst, lane & 1);
+            bulk_commit();
+          }
+          if (lane < 2) bulk_wait_read_all();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.dst_free);
+        }
+        if (lane < 4) bulk_wait_read_all();
+        __syncwarp();
+        if (lane == 0) {
           mbar_arrive(&S.kvst_free);
           mbar_arrive(&S.sched_empty[sl]);
-          ++n;
         }
-        if (ok && gt > 0 && !reduce_dq(gt - 1)) ok = false;
-        if (!ok) fail();
-        bulk_wait_all();
+        ++n;
       }
+      if (ok && gt > 0 && !reduce_dq(gt - 1)) ok = false;
+      if (!ok && lane == 0) fail();
+      bulk_wait_all();
     }
   } else {
     regs_increase<kRegsCompute>();
