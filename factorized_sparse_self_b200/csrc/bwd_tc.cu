@@ -258,6 +258,10 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  if (warp == 11) {  // the tensor maps into the descriptor cache, one per lane
+    const CUtensorMap* m = &maps.q[0];
+    if (lane < (int)(sizeof(BwdMaps) / sizeof(CUtensorMap))) tma_prefetch_desc(m + lane);
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;

@@ -186,6 +186,10 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  if (warp == 7) {  // the tensor maps into the descriptor cache, one per lane
+    const CUtensorMap* m = &maps.q[0];
+    if (lane < (int)(sizeof(FwdMaps) / sizeof(CUtensorMap))) tma_prefetch_desc(m + lane);
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
