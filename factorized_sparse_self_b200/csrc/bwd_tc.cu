@@ -71,6 +71,14 @@ struct SchedSlot {
   QEnt q[kBwdChunk];
 };
 
+// Natural rows of each head class whose gradient no unit writes (zero),
+// for dQ and for dK / dV.
+struct ZeroRows {
+  const int32_t* q[2];
+  const int32_t* k[2];
+  int32_t nq[2], nk[2];
+};
+
 struct SmemBwd {
   uint8_t k[2][kTileBytes];
   uint8_t v[2][kTileBytes];
@@ -209,8 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __restrict__ items,
               int n_units, int NH, const QEnt* __restrict__ qents, Heads hs,
               float scale, float scale_log2, const float* __restrict__ lse,
-              const float* __restrict__ Dg, int* sched_counter, int* status,
-              uint64_t wait_ns) {
+              const float* __restrict__ Dg, ZeroRows zr, uint4* __restrict__ dq_out,
+              uint4* __restrict__ dk_out, uint4* __restrict__ dv_out, int* sched_counter,
+              int* status, uint64_t wait_ns) {
   // The shared-memory plan fills the 227 KB a CTA may hold, with no room to
   // realign: the swizzled tiles need the dynamic window at a 1024-byte
   // boundary (where it starts when the kernel has no static shared memory).
@@ -582,6 +591,33 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       if (ok && gt > 0 && !reduce_dq(gt - 1)) ok = false;
       if (!ok && lane == 0) fail();
       bulk_wait_all();
+    } else if (warp == 11) {
+      // ---------------- zero-fill of the rows no unit writes ----------------
+      // (their gradient is zero), in the background of the other roles. Work
+      // items of 128 listed rows of one head are spread over the CTAs; eight
+      // lanes cover a 128-byte row, four rows per step.
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      const int nheads = hs.B * hs.hn;
+      for (int pass = 0; pass < 2; ++pass) {
+        const int most = pass ? max(zr.nk[0], zr.nk[1]) : max(zr.nq[0], zr.nq[1]);
+        const int chunks = (most + 127) / 128;
+        const int items_total = nheads * chunks;
+        for (int w = blockIdx.x; w < items_total; w += gridDim.x) {
+          const int x = w / chunks, ck = w - x * chunks;
+          const int bh = (x / hs.hn) * hs.H + hs.h0 + x % hs.hn;
+          const int hc = class_of(bh, hs);
+          const int n = pass ? (hc ? zr.nk[1] : zr.nk[0]) : (hc ? zr.nq[1] : zr.nq[0]);
+          const int32_t* rows = pass ? (hc ? zr.k[1] : zr.k[0]) : (hc ? zr.q[1] : zr.q[0]);
+          const int r1 = min(n, ck * 128 + 128);
+          uint4* base0 = (pass ? dk_out : dq_out) + (size_t)bh * g.T * 8 + (lane & 7);
+          uint4* base1 = dv_out + (size_t)bh * g.T * 8 + (lane & 7);
+          for (int r = ck * 128 + (lane >> 3); r < r1; r += 4) {
+            const size_t at = (size_t)rows[r] * 8;
+            base0[at] = z;
+            if (pass) base1[at] = z;
+          }
+        }
+      }
     }
   } else {
     regs_increase<kRegsCompute>();
@@ -827,11 +863,18 @@ cudaError_t tc_bwd_t(const Call& c, const void* q, const void* k, const void* v,
   const long long units = (long long)L->dev.n_bwd_split[f] * NH;
   if (units > 0x7fffffff) return cudaErrorInvalidValue;
   const int grid = (int)std::min<long long>(units, sms);
+  ZeroRows zr;
+  for (int hc = 0; hc < 2; ++hc) {
+    zr.q[hc] = (const int32_t*)L->dev.rows[hc][ROWS_Q_ZERO];
+    zr.k[hc] = (const int32_t*)L->dev.rows[hc][ROWS_K_ZERO];
+    zr.nq[hc] = L->dev.n_rows[hc][ROWS_Q_ZERO];
+    zr.nk[hc] = L->dev.n_rows[hc][ROWS_K_ZERO];
+  }
   record_begin(c);
   bwd_tc_kernel<F16><<<grid, kThreads, smem, c.stream>>>(
       maps, L->geom, (const BwdItem*)L->dev.bwd_split[f], (int)units, NH,
       (const QEnt*)L->dev.q_ents, heads_of(c), c.scale, c.scale * kLog2e, lse, D,
-      sched_counter, c.status,
+      zr, (uint4*)dq, (uint4*)dk, (uint4*)dv, sched_counter, c.status,
       c.wait_ns);
   err = cudaGetLastError();
   record_end(c);

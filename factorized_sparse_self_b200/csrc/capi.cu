@@ -369,7 +369,7 @@ st_status st_sparse_attn_bwd_heads(const st_layout* L, st_dtype dtype, int32_t B
     float* dk_acc = acc + stride;
     float* dv_acc = acc + 2 * stride;
     int* counter = reinterpret_cast<int*>(dv_acc + stride);  // work counter of the kernel
-    e = bwd_prep(c, o, dout, Dv, dq_acc, dk_acc, dv_acc, dq, dk, dv, counter);
+    e = bwd_prep(c, o, dout, Dv, dq_acc, dk_acc, dv_acc, counter);
     Call cm = c;
     arm(cm, 1);
     if (e == cudaSuccess)

@@ -323,8 +323,7 @@ __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __rest
                                 float* __restrict__ Dv,
                                 int T, Heads hs, RowSet rs, float4* __restrict__ dq_acc,
                                 float4* __restrict__ dk_acc, float4* __restrict__ dv_acc,
-                                uint4* __restrict__ dq, uint4* __restrict__ dk,
-                                uint4* __restrict__ dv, int* __restrict__ sched_counter) {
+                                int* __restrict__ sched_counter) {
   // grid.y runs over the selected heads of every batch
   const int bh = (blockIdx.y / hs.hn) * hs.H + hs.h0 + blockIdx.y % hs.hn;
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *sched_counter = 0;
@@ -362,7 +361,6 @@ __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __rest
     }
   }
   const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-  const uint4 zu = make_uint4(0u, 0u, 0u, 0u);
   {
     int nr;
     const int32_t* rows = rows_of(rs, hc, ROWS_Q_ACC, nr);
@@ -376,21 +374,6 @@ __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __rest
       const size_t e = (rb + rows[x >> 4]) * 16 + (x & 15);
       dk_acc[e] = z4;
       dv_acc[e] = z4;
-    }
-  }
-  {
-    int nr;
-    const int32_t* rows = rows_of(rs, hc, ROWS_Q_ZERO, nr);
-    for (int64_t x = tid; x < (int64_t)nr * 8; x += stride)
-      dq[(rb + rows[x >> 3]) * 8 + (x & 7)] = zu;
-  }
-  {
-    int nr;
-    const int32_t* rows = rows_of(rs, hc, ROWS_K_ZERO, nr);
-    for (int64_t x = tid; x < (int64_t)nr * 8; x += stride) {
-      const size_t e = (rb + rows[x >> 3]) * 8 + (x & 7);
-      dk[e] = zu;
-      dv[e] = zu;
     }
   }
 }
@@ -549,16 +532,14 @@ cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* 
 }
 
 cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* Dv, float* dq_acc,
-                     float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv,
-                     int* sched_counter) {
+                     float* dk_acc, float* dv_acc, int* sched_counter) {
   const int T = c.L->geom.T;
   const int bx = std::max(1, std::min(64, (T + 127) / 128));
   dim3 grid(bx, c.B * c.hn);
   auto kern = (c.dtype == ST_F16) ? bwd_prep_kernel<true> : bwd_prep_kernel<false>;
   kern<<<grid, 256, 0, c.stream>>>(
       (const uint4*)o, (const uint4*)dout, Dv, T, heads_of(c),
-      row_set_of(c.L), (float4*)dq_acc, (float4*)dk_acc, (float4*)dv_acc, (uint4*)dq, (uint4*)dk,
-      (uint4*)dv, sched_counter);
+      row_set_of(c.L), (float4*)dq_acc, (float4*)dk_acc, (float4*)dv_acc, sched_counter);
   return cudaGetLastError();
 }
 

@@ -45,16 +45,14 @@ cudaError_t simt_bwd(const Call& c, const void* q, const void* k, const void* v,
 cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* D, float* acc,
                          size_t acc_elems);
 
-// bf16 backward, around the tensor-core kernel: bwd_prep writes D for every
-// row, zeroes the fp32 accumulator rows that collect several contributions and
-// zero-fills the output rows nobody writes; bwd_finish rounds the accumulated
-// rows into dq, dk, dv (scale applied to dQ and dK). Rows that a single
-// backward unit produces are written by the tensor-core kernel itself.
-// bwd_prep also zeroes the work counter the tensor-core kernel claims its
-// units from.
+// 16-bit backward, around the tensor-core kernel: bwd_prep writes D for every
+// row and zeroes the fp32 accumulator rows that collect several contributions
+// and the work counter the tensor-core kernel claims its units from;
+// bwd_finish rounds the accumulated rows into dq, dk, dv (scale applied to dQ
+// and dK). Rows that a single backward unit produces, and rows nobody writes
+// (zero-filled), are written by the tensor-core kernel itself.
 cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* D, float* dq_acc,
-                     float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv,
-                     int* sched_counter);
+                     float* dk_acc, float* dv_acc, int* sched_counter);
 cudaError_t bwd_finish(const Call& c, const float* dq_acc, const float* dk_acc,
                        const float* dv_acc, void* dq, void* dk, void* dv);
 
