@@ -699,11 +699,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&S.sdp_free);  // S^T, dP^T of this tile may now be overwritten
-        if (!full) {
-#pragma unroll
-          for (int xk = 0; xk < 64; ++xk)
-            if (wg * 64 + xk < lo || wg * 64 + xk >= hi) sv[xk] = -INFINITY;
-        }
+        if (!full) mask_cols<2>(sv, wg * 64, lo, hi);
         const float* l2 = S.l2[s] + wg * 64;
         const float* dd = S.dd[s] + wg * 64;
         // P^T and dS^T of the whole row slice in registers first: the tensor

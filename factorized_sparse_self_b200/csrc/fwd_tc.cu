@@ -93,10 +93,10 @@ __device__ __forceinline__ void prefetch_tile(const CUtensorMap* maps, int view,
 }
 
 // Live key columns [lo, hi) of key tile `ke` for the query at natural
-// position i (and, in the residue view, its class row p = i / l). The bounds
-// restate the segment rules as intervals.
-__device__ __forceinline__ void live_cols(const Geom& g, const KeyEnt& ke, int i, int& lo,
-                                          int& hi) {
+// position i, with blk = i / l (its block, or in the residue view its class
+// row). The bounds restate the segment rules as intervals.
+__device__ __forceinline__ void live_cols(const Geom& g, const KeyEnt& ke, int i, int blk,
+                                          int& lo, int& hi) {
   if (i < 0) {
     lo = hi = 0;
     return;
@@ -109,7 +109,7 @@ __device__ __forceinline__ void live_cols(const Geom& g, const KeyEnt& ke, int i
     switch (ke.rule) {
       case RULE_CAUSAL: a = 0; b = i + 1; break;
       case RULE_BAND: a = max(0, i - l); b = i + 1; break;
-      case RULE_BLOCK: a = (i / l) * l; b = i + 1; break;
+      case RULE_BLOCK: a = blk * l; b = i + 1; break;
       case RULE_STRIDE: a = i; b = i + 1; break;          // natural keys only when l >= T
       case RULE_SUMMARY: a = l - c; b = i + 1; break;     // natural keys only when l >= T
       default: a = 0; b = 0; break;                        // stride_far / summary_earlier: empty
@@ -117,16 +117,15 @@ __device__ __forceinline__ void live_cols(const Geom& g, const KeyEnt& ke, int i
   } else if (ke.kview == VIEW_SUM) {
     base = ke.ktile * kTile;
     lim = g.nsum;
-    const int blk = i / l, off = i - blk * l;
+    const int off = i - blk * l;
     a = 0;
     b = blk * c + ((ke.rule == RULE_SUMMARY) ? max(0, off - (l - c) + 1) : 0);
   } else {
     const int pb = ke.ktile % g.ptiles;
     base = pb * kTile;
     lim = g.P;
-    const int p = i / l;
     a = 0;
-    b = (ke.rule == RULE_STRIDE) ? p + 1 : p - 1;
+    b = (ke.rule == RULE_STRIDE) ? blk + 1 : blk - 1;
   }
   b = min(b, lim);
   lo = max(a - base, 0);
@@ -500,12 +499,24 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           }
         }
       }
+      // the row leaves in whole 32-byte sectors when the output allows it
+      // (rows are 128 bytes, so all rows share the base's alignment)
+      if ((reinterpret_cast<uintptr_t>(out) & 31) == 0) {
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        dst[ch] = make_uint4(pack2<F16>(o[ch * 8 + 0], o[ch * 8 + 1]),
-                             pack2<F16>(o[ch * 8 + 2], o[ch * 8 + 3]),
-                             pack2<F16>(o[ch * 8 + 4], o[ch * 8 + 5]),
-                             pack2<F16>(o[ch * 8 + 6], o[ch * 8 + 7]));
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t w[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) w[x] = pack2<F16>(o[ch * 16 + 2 * x], o[ch * 16 + 2 * x + 1]);
+          st_global_v8(dst + 2 * ch, w);
+        }
+      } else {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          dst[ch] = make_uint4(pack2<F16>(o[ch * 8 + 0], o[ch * 8 + 1]),
+                               pack2<F16>(o[ch * 8 + 2], o[ch * 8 + 3]),
+                               pack2<F16>(o[ch * 8 + 4], o[ch * 8 + 5]),
+                               pack2<F16>(o[ch * 8 + 6], o[ch * 8 + 7]));
+      }
       lse[(size_t)pe.bh * g.T + pe.i] = L;
     };
     auto epilogue = [&](const Pending& pe) {
@@ -527,6 +538,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       const FwdItem& it = x.it;
       const int bh = x.bh;
       const int i = view_pos(g, it.qview, it.qtile, row);
+      const int iblk = i >= 0 ? i / g.l : 0;
       const int cnt = it.kend - it.kbeg;
       if (cnt == 0) {
         if (pending) {
@@ -560,10 +572,8 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         const bool full = (ke.flag == TILE_FULL);
         if (!full) {
           int lo, hi;
-          live_cols(g, ke, i, lo, hi);
-#pragma unroll
-          for (int xk = 0; xk < 128; ++xk)
-            if (xk < lo || xk >= hi) s[xk] = -INFINITY;
+          live_cols(g, ke, i, iblk, lo, hi);
+          mask_cols<4>(s, 0, lo, hi);
         }
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll

@@ -405,6 +405,13 @@ __device__ __forceinline__ float2 unpack2(uint32_t u) {
     return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
 }
 
+// 32-byte global store (the address must be 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
@@ -418,6 +425,24 @@ __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_
                : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
                : "r"(addr)
                : "memory");
+}
+
+// Sets v[x] = -inf for the columns base + x (x < 32 * NCHUNK) outside this
+// row's live interval [lo, hi). A chunk of 32 columns that every row of the
+// warp keeps is skipped (warp-uniform branch); the others are selected
+// element by element.
+template <int NCHUNK>
+__device__ __forceinline__ void mask_cols(float* v, int base, int lo, int hi) {
+  const unsigned span = (unsigned)(hi - lo);
+#pragma unroll
+  for (int ch = 0; ch < NCHUNK; ++ch) {
+    const int c0 = base + ch * 32;
+    if (!__all_sync(0xffffffffu, lo <= c0 && hi >= c0 + 32)) {
+#pragma unroll
+      for (int x = 0; x < 32; ++x)
+        v[ch * 32 + x] = ((unsigned)(c0 + x - lo) < span) ? v[ch * 32 + x] : -INFINITY;
+    }
+  }
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {

@@ -113,6 +113,26 @@ def test_forward_is_deterministic_and_guard_regions_untouched():
     assert (lbuf[:pad] == 3.0).all() and (lbuf[-pad:] == 3.0).all()
 
 
+def test_forward_output_16_byte_aligned_matches_aligned():
+    """O rows are stored 32 bytes at a time when the output allows it; an
+    output that is only 16-byte aligned (the ABI's minimum) takes the 16-byte
+    stores and must give the same bits, without touching its neighbours."""
+    B, H, T, d = 1, 2, 1024, 64
+    (_, _, _, _), (qd, kd, vd, _) = device_inputs(B, H, T, d, "bf16", 0.5)
+    L = st.st_pattern_layout("fixed", "merged", T, 128, 8)
+    o_ref, lse_ref = st.st_sparse_attn_fwd(L, qd, kd, vd)
+    pad = 8  # 16 bytes of bf16
+    n = B * H * T * d
+    buf = torch.full((n + 2 * pad,), 5.0, dtype=torch.bfloat16, device="cuda")
+    o = buf[pad:pad + n].view(B, H, T, d)
+    assert o.data_ptr() % 32 == 16
+    _, lse = st.st_sparse_attn_fwd(L, qd, kd, vd, o=o)
+    torch.cuda.synchronize()
+    assert st.st_last_device_status() == st.ST_OK
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+    assert (buf[:pad] == 5.0).all() and (buf[-pad:] == 5.0).all()
+
+
 def test_bad_arguments_rejected_before_launch():
     L = st.st_pattern_layout("fixed", "split", 1024, 64, 8)
     q = torch.zeros(1, 2, 1024, 64, dtype=torch.bfloat16, device="cuda")
