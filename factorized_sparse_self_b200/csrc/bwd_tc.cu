@@ -395,13 +395,24 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         };
         if (kv_last < n) ok = load_kv(n, x);
         if (!ok) break;
-        if (cnt > 0) ok = issue_q(0);
-        const int nxt = valid((int)gridDim.x + __shfl_sync(0xffffffffu, ticket, 0));
-        if (ok && cnt > 1) ok = issue_q(1);
-        // the following unit's K, V as soon as unit n - 1 has released their
-        // buffer: by now its last tiles have passed through the ring
-        if (ok && nxt < n_units) ok = load_kv(n + 1, unit_of(items, nxt, NH, hs));
-        for (int e = 2; ok && e < cnt; ++e) ok = issue_q(e);
+        // Q, dO of the unit's query tiles in order; the claimed next unit is
+        // resolved after the first, and its K, V go out after the second (or
+        // after the last, for shorter units), as soon as unit n - 1 has
+        // released their buffer. One call site per loader keeps the warp's
+        // code small.
+        int nxt = n_units;
+        bool kv_next = false;
+        for (int e = 0; ok; ++e) {
+          if (e < cnt) ok = issue_q(e);
+          if (!ok) break;
+          if (e == 0) nxt = valid((int)gridDim.x + __shfl_sync(0xffffffffu, ticket, 0));
+          const bool last = e + 1 >= cnt;
+          if (!kv_next && (e == 1 || last)) {
+            kv_next = true;
+            if (nxt < n_units) ok = load_kv(n + 1, unit_of(items, nxt, NH, hs));
+          }
+          if (last && kv_next) break;
+        }
         ++n;
         cur = nxt;
       }

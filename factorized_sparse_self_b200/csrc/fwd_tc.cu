@@ -145,7 +145,11 @@ __device__ __forceinline__ Unit unit_of(const FwdItem* items, int u, int NH, con
   return x;
 }
 
-template <bool F16>  // 16-bit element type: fp16 if true, else bf16
+// F16: 16-bit element type (fp16 if true, else bf16). MERGE: the launch is
+// the second pass of a two-pass layout and merges its result into the O and
+// LSE already in the outputs (a separate instantiation, so that one-pass
+// launches carry no merge code).
+template <bool F16, bool MERGE>
 __global__ void __launch_bounds__(kThreads, 2)
 fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __restrict__ items,
               int n_units, int NH, const KeyEnt* __restrict__ keys, Heads hs,
@@ -477,7 +481,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       for (int xk = 0; xk < 64; ++xk) o[xk] *= inv;
       const size_t rowoff = ((size_t)pe.bh * g.T + pe.i) * 64;
       uint4* dst = reinterpret_cast<uint4*>(out + rowoff);
-      if (pe.merge) {
+      if constexpr (MERGE) {
         const float Lp = lse[(size_t)pe.bh * g.T + pe.i];
         const float mx2 = fmaxf(Lp, L);
         float wp = 0.f, wc = 0.f;
@@ -533,23 +537,31 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         ok = false;
         break;
       }
-      if (u >= n_units) break;
-      const Unit x = unit_of(items, u, NH, hs);
+      const bool end = u >= n_units;
+      Unit x;
+      x.it = FwdItem{0, 0, 0, 0, 0, 0, 0};
+      x.bh = 0;
+      if (!end) x = unit_of(items, u, NH, hs);
       const FwdItem& it = x.it;
-      const int bh = x.bh;
-      const int i = view_pos(g, it.qview, it.qtile, row);
+      const int i = end ? -1 : view_pos(g, it.qview, it.qtile, row);
       const int iblk = i >= 0 ? i / g.l : 0;
       const int cnt = it.kend - it.kbeg;
-      if (cnt == 0) {
+      if (end || cnt == 0) {
+        // the pending unit's output goes out here (one copy of the epilogue
+        // for empty units and for the end of the work); an empty unit then
+        // becomes the pending one, written by the next flush
         if (pending) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&S.pv_done, (gt - 1) & 1, wait_ns, abort));
-          if (!ok) break;
-          tc_fence_after();
+          if (gt > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&S.pv_done, (gt - 1) & 1, wait_ns, abort));
+            if (!ok) break;
+            tc_fence_after();
+          }
           epilogue(pend);
           pending = false;
         }
-        const Pending z = {i, bh, 0, (int)it.merge, -INFINITY, 0.f};
-        epilogue(z);
+        if (end) break;
+        pend = {i, x.bh, 0, (int)it.merge, -INFINITY, 0.f};
+        pending = true;
         ++n;
         continue;
       }
@@ -645,16 +657,9 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         }
       }
       if (!ok) break;
-      pend = {i, bh, cnt, (int)it.merge, m_run, l_run};
+      pend = {i, x.bh, cnt, (int)it.merge, m_run, l_run};
       pending = true;
       ++n;
-    }
-    if (ok && pending) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&S.pv_done, (gt - 1) & 1, wait_ns, abort));
-      if (ok) {
-        tc_fence_after();
-        epilogue(pend);
-      }
     }
     if (!ok) fail();
   }
@@ -692,8 +697,11 @@ cudaError_t tc_fwd_t(const Call& c, const void* q, const void* k, const void* v,
   cudaGetDevice(&dev);
   cudaError_t err = cudaSuccess;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    err = cudaFuncSetAttribute(fwd_tc_kernel<F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
+    err = cudaFuncSetAttribute(fwd_tc_kernel<F16, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(fwd_tc_kernel<F16, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
@@ -708,7 +716,9 @@ cudaError_t tc_fwd_t(const Call& c, const void* q, const void* k, const void* v,
     const long long units = (long long)n * NH;
     if (units > 0x7fffffff) return cudaErrorInvalidValue;
     const int grid = (int)std::min<long long>(units, 2LL * sms);
-    fwd_tc_kernel<F16><<<grid, kThreads, smem, c.stream>>>(
+    // the second pass of a two-pass layout merges into the first's O, LSE
+    auto kernel = pass > 0 ? fwd_tc_kernel<F16, true> : fwd_tc_kernel<F16, false>;
+    kernel<<<grid, kThreads, smem, c.stream>>>(
         maps, L->geom, (const FwdItem*)L->dev.fwd_items[pass], (int)units, NH,
         (const KeyEnt*)L->dev.key_ents, heads_of(c), scale_log2, (uint16_t*)o, lse,
         slot, c.status, c.wait_ns, (force_timeout && pass == 0) ? 1 : 0);
