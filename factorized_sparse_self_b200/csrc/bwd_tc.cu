@@ -301,22 +301,23 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       // The CTA's first unit is blockIdx.x (the longest units spread one per
       // CTA); later ones come from the counter, offset by the grid. Units
       // without a head of their class are skipped.
-      auto valid = [&](int u) -> int {
+      // The first valid unit at or after u (n_units if none), decoded into y.
+      auto valid = [&](int u, Unit& y) -> int {
         for (;;) {
           if (u >= n_units) return n_units;
-          if (unit_of(items, u, NH, hs).bh >= 0) return u;
+          y = unit_of(items, u, NH, hs);
+          if (y.bh >= 0) return u;
           int t = 0;
           if (lane == 0) t = atomicAdd(sched_counter, 1);
           u = (int)gridDim.x + __shfl_sync(0xffffffffu, t, 0);
         }
       };
-      auto publish = [&](int u) -> bool {
+      auto publish = [&](int u, const Unit& x) -> bool {
         const int k = pub % kSched;
         const bool w = mbar_wait(&S.sched_empty[k], ((pub / kSched) & 1) ^ 1, wait_ns, abort);
         if (!__all_sync(0xffffffffu, w)) return false;
         SchedSlot& sl = S.slot[k];
         if (u < n_units) {
-          const Unit x = unit_of(items, u, NH, hs);
           if (lane < x.it.qend - x.it.qbeg) sl.q[lane] = qents[x.it.qbeg + lane];
           if (lane == 0) {
             sl.bh = x.bh;
@@ -329,15 +330,15 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         ++pub;
         return true;
       };
-      int cur = valid(blockIdx.x);
+      Unit x;
+      int cur = valid(blockIdx.x, x);
       while (ok && cur < n_units) {
-        ok = publish(cur);
+        ok = publish(cur, x);
         if (!ok) break;
         // the claim of the following unit goes out now; its answer is first
         // needed once this unit's K, V are on their way
         int ticket = 0;
         if (lane == 0) ticket = atomicAdd(sched_counter, 1);
-        const Unit x = unit_of(items, cur, NH, hs);
         const int cnt = x.it.qend - x.it.qbeg;
         auto issue_q = [&](int e) -> bool {
           const int s = gt % NS;
@@ -401,22 +402,24 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         // released their buffer. One call site per loader keeps the warp's
         // code small.
         int nxt = n_units;
+        Unit y;
         bool kv_next = false;
         for (int e = 0; ok; ++e) {
           if (e < cnt) ok = issue_q(e);
           if (!ok) break;
-          if (e == 0) nxt = valid((int)gridDim.x + __shfl_sync(0xffffffffu, ticket, 0));
+          if (e == 0) nxt = valid((int)gridDim.x + __shfl_sync(0xffffffffu, ticket, 0), y);
           const bool last = e + 1 >= cnt;
           if (!kv_next && (e == 1 || last)) {
             kv_next = true;
-            if (nxt < n_units) ok = load_kv(n + 1, unit_of(items, nxt, NH, hs));
+            if (nxt < n_units) ok = load_kv(n + 1, y);
           }
           if (last && kv_next) break;
         }
         ++n;
         cur = nxt;
+        x = y;
       }
-      if (ok) ok = publish(n_units);  // no more work
+      if (ok) ok = publish(n_units, x);  // no more work
       if (!ok && lane == 0) fail();
       if (lane == 0) {
         // the last K / V loads of both buffers have landed before the exit
@@ -466,17 +469,22 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           k_addr = smem_u32(S.k[kb]);
           v_addr = smem_u32(S.v[kb]);
           ok = mbar_wait(&S.kv_full[kb], (n >> 1) & 1, wait_ns, abort);
-          if (ok) ok = issue_s_dp(gt);
-          for (int e = 0; ok && e < cnt; ++e, ++gt) {
-            const int s = gt % NS;
-            // S^T, dP^T of the next tile as soon as the compute warps hold this
-            // tile's in registers
+          // e = -1 issues S^T, dP^T of the unit's first tile; tile e issues
+          // those of tile e + 1 as soon as the compute warps hold tile e's in
+          // registers (one issue site)
+          for (int e = -1; ok && e < cnt; gt += (e >= 0), ++e) {
             if (e + 1 < cnt) {
-              if (!mbar_wait(&S.sdp_free, gt & 1, wait_ns, abort) || !issue_s_dp(gt + 1)) {
+              if (e >= 0 && !mbar_wait(&S.sdp_free, gt & 1, wait_ns, abort)) {
+                ok = false;
+                break;
+              }
+              if (!issue_s_dp(e < 0 ? gt : gt + 1)) {
                 ok = false;
                 break;
               }
             }
+            if (e < 0) continue;
+            const int s = gt % NS;
             if (!mbar_wait(&S.ds_ready, gt & 1, wait_ns, abort)) {
               ok = false;
               break;
@@ -552,23 +560,27 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           ok = false;
           break;
         }
-        if (u >= n_units) break;
+        const bool end = u >= n_units;
         Unit x;
         x.it = S.slot[sl].it;
         x.bh = S.slot[sl].bh;
-        const int cnt = x.it.qend - x.it.qbeg;
+        // the dQ of each tile goes out while the next is computed; the end of
+        // the work is one more step that only sends the last tile's (one call
+        // site)
+        const int cnt = end ? 1 : x.it.qend - x.it.qbeg;
         for (int e = 0; ok && e < cnt; ++e, ++gt) {
           if (gt > 0 && !reduce_dq(gt - 1)) {
             ok = false;
             break;
           }
+          if (end) break;
           const QEnt qe = S.slot[sl].q[e];
           pv = x.it.qview;
           ptile = qe.qtile;
           pdirect = qe.q_direct;
           pbh = x.bh;
         }
-        if (!ok) break;
+        if (!ok || end) break;
         const bool w = mbar_wait(&S.out_full, n & 1, wait_ns, abort);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
@@ -599,7 +611,6 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         }
         ++n;
       }
-      if (ok && gt > 0 && !reduce_dq(gt - 1)) ok = false;
       if (!ok && lane == 0) fail();
       bulk_wait_all();
     } else if (warp == 11) {

@@ -227,10 +227,12 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       int n = 0, pub = 0;
       // Unit u of the CTA's first is blockIdx.x (the longest units spread one
       // per CTA); later ones come from the counter, offset by the grid.
-      auto valid = [&](int u) -> int {
+      // The first valid unit at or after u (n_units if none), decoded into y.
+      auto valid = [&](int u, Unit& y) -> int {
         for (;;) {
           if (u >= n_units) return n_units;
-          if (unit_of(items, u, NH, hs).bh >= 0) return u;
+          y = unit_of(items, u, NH, hs);
+          if (y.bh >= 0) return u;
           u = (int)gridDim.x + atomicAdd(sched_slot, 1);
         }
       };
@@ -242,7 +244,8 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         ++pub;
         return true;
       };
-      int cur = valid(blockIdx.x);
+      Unit x;
+      int cur = valid(blockIdx.x, x);
       while (ok && cur < n_units) {
         if (!publish(cur)) {
           ok = false;
@@ -250,7 +253,6 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         }
         // the claim of the following unit goes out now, answered by the end
         const int ticket = (int)gridDim.x + atomicAdd(sched_slot, 1);
-        const Unit x = unit_of(items, cur, NH, hs);
         const int qb = n & 1;
         if (!mbar_wait(&S.q_empty[qb], ((n >> 1) & 1) ^ 1, wait_ns, abort)) {
           ok = false;
@@ -276,7 +278,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           kv_last[s] = gt;
         }
         ++n;
-        cur = valid(ticket);
+        cur = valid(ticket, x);
       }
       if (ok && !publish(n_units)) ok = false;  // no more work
       if (!ok) fail();
