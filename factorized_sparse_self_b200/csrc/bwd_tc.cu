@@ -103,9 +103,9 @@ __device__ __forceinline__ void load_tile(void* dst, const CUtensorMap* maps, in
   if (view == VIEW_NAT) {
     tma_load_3d(dst, &maps[VIEW_NAT], bar, 0, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
-    tma_load_4d(dst, &maps[VIEW_SUM], bar, 0, g.l - g.c, tile * (kTile / g.c), bh);
+    tma_load_4d(dst, &maps[VIEW_SUM], bar, 0, g.l - g.c, tile * g.sum_rows, bh);
   } else {
-    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+    int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_load_4d(dst, &maps[VIEW_CLS], bar, 0, r, pb * kTile, bh);
   }
 }
@@ -116,9 +116,9 @@ __device__ __forceinline__ void prefetch_tile(const CUtensorMap* maps, int view,
   if (view == VIEW_NAT) {
     tma_prefetch_3d(&maps[VIEW_NAT], 0, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
-    tma_prefetch_4d(&maps[VIEW_SUM], 0, g.l - g.c, tile * (kTile / g.c), bh);
+    tma_prefetch_4d(&maps[VIEW_SUM], 0, g.l - g.c, tile * g.sum_rows, bh);
   } else {
-    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+    int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_prefetch_4d(&maps[VIEW_CLS], 0, r, pb * kTile, bh);
   }
 }
@@ -133,9 +133,9 @@ __device__ __forceinline__ void reduce_half(const CUtensorMap* maps, int view, c
   if (view == VIEW_NAT) {
     tma_reduce_add_3d(&maps[VIEW_NAT], s, h * 32, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
-    tma_reduce_add_4d(&maps[VIEW_SUM], s, h * 32, g.l - g.c, tile * (kTile / g.c), bh);
+    tma_reduce_add_4d(&maps[VIEW_SUM], s, h * 32, g.l - g.c, tile * g.sum_rows, bh);
   } else {
-    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+    int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_reduce_add_4d(&maps[VIEW_CLS], s, h * 32, r, pb * kTile, bh);
   }
 }
@@ -146,9 +146,9 @@ __device__ __forceinline__ void store_tile(const CUtensorMap* maps, int view, co
   if (view == VIEW_NAT) {
     tma_store_3d(&maps[VIEW_NAT], src, 0, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
-    tma_store_4d(&maps[VIEW_SUM], src, 0, g.l - g.c, tile * (kTile / g.c), bh);
+    tma_store_4d(&maps[VIEW_SUM], src, 0, g.l - g.c, tile * g.sum_rows, bh);
   } else {
-    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+    int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_store_4d(&maps[VIEW_CLS], src, 0, r, pb * kTile, bh);
   }
 }
@@ -170,28 +170,28 @@ __device__ __forceinline__ void live_rows(const Geom& g, int kview, int qview, i
     return;
   }
   const int l = g.l, c = g.c;
+  const int jb = fdiv(j, g.fl);  // the key's block (its class row in the residue view)
   int a = 0, b = 0, base, lim;
   if (qview == VIEW_NAT) {
     base = qtile * kTile;
     lim = g.T;
     if (kview == VIEW_SUM) {
-      a = (rule == RULE_SUMMARY) ? j : (j / l + 1) * l;
+      a = (rule == RULE_SUMMARY) ? j : (jb + 1) * l;
       b = lim;
     } else {
       switch (rule) {
         case RULE_CAUSAL: a = j; b = lim; break;
         case RULE_BAND: a = j; b = j + l + 1; break;
-        case RULE_BLOCK: a = j; b = (j / l + 1) * l; break;
+        case RULE_BLOCK: a = j; b = (jb + 1) * l; break;
         case RULE_STRIDE: a = j; b = j + 1; break;                          // l >= T only
-        case RULE_SUMMARY: a = j; b = (j % l >= l - c) ? lim : j; break;    // l >= T only
+        case RULE_SUMMARY: a = j; b = (j - jb * l >= l - c) ? lim : j; break;  // l >= T only
         default: a = 0; b = 0; break;
       }
     }
   } else {
-    base = (qtile % g.ptiles) * kTile;
+    base = (qtile - fdiv(qtile, g.fpt) * g.ptiles) * kTile;
     lim = g.P;
-    const int pk = j / l;
-    a = (rule == RULE_STRIDE) ? pk : pk + 2;
+    a = (rule == RULE_STRIDE) ? jb : jb + 2;
     b = lim;
   }
   b = min(b, lim);
@@ -207,8 +207,9 @@ struct Unit {
 
 __device__ __forceinline__ Unit unit_of(const BwdItem* items, int u, int NH, const Heads& hs) {
   Unit x;
-  x.it = items[u / NH];
-  x.bh = head_of(u % NH, x.it.hclass, hs);
+  const int q = fdiv(u, hs.fnh);  // NH = the divisor of hs.fnh
+  x.it = items[q];
+  x.bh = head_of(u - q * NH, x.it.hclass, hs);
   return x;
 }
 
@@ -626,7 +627,8 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         const int items_total = nheads * chunks;
         for (int w = blockIdx.x; w < items_total; w += gridDim.x) {
           const int x = w / chunks, ck = w - x * chunks;
-          const int bh = (x / hs.hn) * hs.H + hs.h0 + x % hs.hn;
+          const int xb = fdiv(x, hs.fhn);
+          const int bh = xb * hs.H + hs.h0 + (x - xb * hs.hn);
           const int hc = class_of(bh, hs);
           const int n = pass ? (hc ? zr.nk[1] : zr.nk[0]) : (hc ? zr.nq[1] : zr.nq[0]);
           const int32_t* rows = pass ? (hc ? zr.k[1] : zr.k[0]) : (hc ? zr.q[1] : zr.q[0]);

@@ -11,6 +11,12 @@
 
 namespace st {
 
+// floor(n / d) for 0 <= n < 2^31, with f = make_fastdiv(d).
+__device__ __forceinline__ int fdiv(int n, FastDiv f) {
+  const uint32_t t = __umulhi(f.m, (uint32_t)n);
+  return (int)((t + (uint32_t)n) >> f.s);
+}
+
 // Natural position of row k of tile `tile` in view v; -1 for padding rows.
 __device__ __forceinline__ int view_pos(const Geom& g, int v, int tile, int k) {
   if (v == VIEW_NAT) {
@@ -20,9 +26,10 @@ __device__ __forceinline__ int view_pos(const Geom& g, int v, int tile, int k) {
   if (v == VIEW_SUM) {
     int s = tile * kTile + k;
     if (s >= g.nsum) return -1;
-    return (s / g.c) * g.l + (g.l - g.c) + s % g.c;
+    const int q = fdiv(s, g.fc);
+    return q * g.l + (g.l - g.c) + (s - q * g.c);
   }
-  int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+  int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
   int p = pb * kTile + k;
   if (p >= g.P) return -1;
   return p * g.l + r;
@@ -63,15 +70,13 @@ __device__ __forceinline__ bool rule_live(const Geom& g, int rule, int i, int j)
 __device__ __forceinline__ int head_of(int x, int hclass, const Heads& hs) {
   if (hs.nclasses == 1) {
     if (x >= hs.B * hs.hn) return -1;
-    const int b = x / hs.hn;
+    const int b = fdiv(x, hs.fhn);
     return b * hs.H + hs.h0 + (x - b * hs.hn);
   }
-  const int first = hs.h0 + ((hclass - hs.h0) & 1);
-  const int end = hs.h0 + hs.hn;
-  const int per = first < end ? (end - 1 - first) / 2 + 1 : 0;
+  const int per = hclass ? hs.per[1] : hs.per[0];
   if (per == 0 || x >= hs.B * per) return -1;
-  const int b = x / per;
-  return b * hs.H + first + 2 * (x - b * per);
+  const int b = fdiv(x, hclass ? hs.fper[1] : hs.fper[0]);
+  return b * hs.H + (hclass ? hs.first[1] : hs.first[0]) + 2 * (x - b * per);
 }
 
 // Head class of flat head index bh (0 for merged layouts).

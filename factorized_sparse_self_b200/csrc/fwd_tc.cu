@@ -72,9 +72,9 @@ __device__ __forceinline__ void load_tile(void* dst, const CUtensorMap* maps, in
   if (view == VIEW_NAT) {
     tma_load_3d(dst, &maps[VIEW_NAT], bar, 0, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
-    tma_load_4d(dst, &maps[VIEW_SUM], bar, 0, g.l - g.c, tile * (kTile / g.c), bh);
+    tma_load_4d(dst, &maps[VIEW_SUM], bar, 0, g.l - g.c, tile * g.sum_rows, bh);
   } else {
-    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+    int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_load_4d(dst, &maps[VIEW_CLS], bar, 0, r, pb * kTile, bh);
   }
 }
@@ -85,9 +85,9 @@ __device__ __forceinline__ void prefetch_tile(const CUtensorMap* maps, int view,
   if (view == VIEW_NAT) {
     tma_prefetch_3d(&maps[VIEW_NAT], 0, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
-    tma_prefetch_4d(&maps[VIEW_SUM], 0, g.l - g.c, tile * (kTile / g.c), bh);
+    tma_prefetch_4d(&maps[VIEW_SUM], 0, g.l - g.c, tile * g.sum_rows, bh);
   } else {
-    int r = tile / g.ptiles, pb = tile - r * g.ptiles;
+    int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_prefetch_4d(&maps[VIEW_CLS], 0, r, pb * kTile, bh);
   }
 }
@@ -121,7 +121,7 @@ __device__ __forceinline__ void live_cols(const Geom& g, const KeyEnt& ke, int i
     a = 0;
     b = blk * c + ((ke.rule == RULE_SUMMARY) ? max(0, off - (l - c) + 1) : 0);
   } else {
-    const int pb = ke.ktile % g.ptiles;
+    const int pb = ke.ktile - fdiv(ke.ktile, g.fpt) * g.ptiles;
     base = pb * kTile;
     lim = g.P;
     a = 0;
@@ -140,8 +140,9 @@ struct Unit {
 
 __device__ __forceinline__ Unit unit_of(const FwdItem* items, int u, int NH, const Heads& hs) {
   Unit x;
-  x.it = items[u / NH];
-  x.bh = head_of(u % NH, x.it.hclass, hs);
+  const int q = fdiv(u, hs.fnh);  // NH = the divisor of hs.fnh
+  x.it = items[q];
+  x.bh = head_of(u - q * NH, x.it.hclass, hs);
   return x;
 }
 
@@ -546,7 +547,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       if (!end) x = unit_of(items, u, NH, hs);
       const FwdItem& it = x.it;
       const int i = end ? -1 : view_pos(g, it.qview, it.qtile, row);
-      const int iblk = i >= 0 ? i / g.l : 0;
+      const int iblk = i >= 0 ? fdiv(i, g.fl) : 0;
       const int cnt = it.kend - it.kbeg;
       if (end || cnt == 0) {
         // the pending unit's output goes out here (one copy of the epilogue

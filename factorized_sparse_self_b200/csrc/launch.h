@@ -70,16 +70,6 @@ cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v,
 
 namespace st {
 
-inline Heads heads_of(const Call& c) {
-  Heads h;
-  h.B = c.B;
-  h.H = c.H;
-  h.h0 = c.h0;
-  h.hn = c.hn;
-  h.nclasses = c.nclasses;
-  return h;
-}
-
 // Units per item: the most heads of one class among the selected heads, times B.
 inline int heads_per_class(const Call& c) {
   if (c.nclasses == 1) return c.B * c.hn;
@@ -90,6 +80,25 @@ inline int heads_per_class(const Call& c) {
     most = std::max(most, first < end ? (end - 1 - first) / 2 + 1 : 0);
   }
   return c.B * most;
+}
+
+inline Heads heads_of(const Call& c) {
+  Heads h;
+  h.B = c.B;
+  h.H = c.H;
+  h.h0 = c.h0;
+  h.hn = c.hn;
+  h.nclasses = c.nclasses;
+  for (int p = 0; p < 2; ++p) {
+    const int first = c.h0 + ((p - c.h0) & 1);
+    const int end = c.h0 + c.hn;
+    h.first[p] = first;
+    h.per[p] = first < end ? (end - 1 - first) / 2 + 1 : 0;
+    h.fper[p] = make_fastdiv(h.per[p]);
+  }
+  h.fhn = make_fastdiv(c.hn);
+  h.fnh = make_fastdiv(heads_per_class(c));
+  return h;
 }
 
 // Element types of tensor maps.

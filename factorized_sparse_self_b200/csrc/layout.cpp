@@ -296,6 +296,10 @@ st_status build_layout(const st_pattern_desc* desc, st_layout* L) {
     g.ptiles = (g.P + kTile - 1) / kTile;
   }
   if (desc->kind == ST_FIXED && has_sum(T, g.l, c)) g.nsum = (int32_t)((T / g.l) * c);
+  g.sum_rows = g.c >= 1 ? kTile / g.c : 0;
+  g.fl = make_fastdiv(g.l);
+  g.fc = make_fastdiv(g.c);
+  g.fpt = make_fastdiv(g.ptiles);
 
   int nhc = (desc->kind != ST_DENSE_CAUSAL && mode == ST_HEADS_SPLIT) ? 2 : 1;
   L->hcs.assign((size_t)nhc, HeadClass());

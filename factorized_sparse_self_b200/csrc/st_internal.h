@@ -86,8 +86,29 @@ enum RowList : int {
 
 // Heads a call covers: heads h0 .. h0+hn-1 of tensors with B x H heads, for a
 // layout with nclasses head classes (kernel parameter, plain old data).
+// Division by a divisor that is fixed for a launch, by a multiply-high and a
+// shift (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994): with s = ceil(log2 d) and m = floor(2^32 (2^s - d)
+// / d) + 1, q = (umulhi(m, n) + n) >> s equals floor(n / d) for every
+// 0 <= n < 2^31 and 1 <= d < 2^31 (the sum stays below 2^32).
+struct FastDiv {
+  uint32_t m, s;
+};
+inline FastDiv make_fastdiv(int32_t d) {
+  if (d < 1) d = 1;  // unused divisors (no such view) get a harmless 1
+  uint32_t s = 0;
+  while ((int64_t(1) << s) < d) ++s;
+  const uint64_t m = ((((uint64_t)1 << s) - (uint64_t)d) << 32) / (uint64_t)d + 1;
+  return FastDiv{(uint32_t)m, s};
+}
+
 struct Heads {
   int32_t B, H, h0, hn, nclasses;
+  // head class p (split layouts): its first head index and heads per batch
+  // entry among h0 .. h0 + hn - 1
+  int32_t first[2], per[2];
+  FastDiv fhn, fper[2];
+  FastDiv fnh;  // units per work item (heads of the largest class, times B)
 };
 
 // Geometry every kernel needs to map view rows to natural positions.
@@ -97,6 +118,8 @@ struct Geom {
   int32_t ptiles;  // 128-row tiles per class, ceil(P / 128)
   int32_t nsum;    // packed summary rows, (T / l) * c (0 when no summary view)
   int32_t kind, mode;
+  int32_t sum_rows;      // summary-view rows of one 128-key tile per l-block, 128 / c
+  FastDiv fl, fc, fpt;   // division by l, c and ptiles
 };
 
 // ---- host-side layout ------------------------------------------------------
