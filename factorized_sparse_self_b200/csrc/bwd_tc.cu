@@ -438,23 +438,24 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         const uint32_t idKM = idesc_16(128, 64, false, true, F16);  // A K-major, B MN-major
         const uint32_t idMM = idesc_16(128, 64, true, true, F16);   // A MN-major, B MN-major
         const uint32_t ds_addr = smem_u32(S.dst);
-        uint32_t k_addr = 0, v_addr = 0;
+        const uint64_t dsk = sdesc(ds_addr, 16, 1024);          // dS^T, K-major (dK)
+        const uint64_t dsm = sdesc(ds_addr, kTileBytes, 1024);  // dS^T read MN-major (dQ)
+        uint64_t kd = 0, vd = 0, kdm = 0;  // this unit's K, V tiles
         bool ok = true;
         int gt = 0, n = 0;
         auto issue_s_dp = [&](int t) -> bool {
           const int s = t % NS;
           if (!mbar_wait(&S.full[s], (t / NS) & 1, wait_ns, abort)) return false;
           tc_fence_after();
-          const uint32_t q_addr = smem_u32(S.q[s]), o_addr = smem_u32(S.dout[s]);
+          const uint64_t qd = sdesc(smem_u32(S.q[s]), 16, 1024);
+          const uint64_t od = sdesc(smem_u32(S.dout[s]), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + kColS, sdesc(k_addr + kk * 32, 16, 1024),
-                   sdesc(q_addr + kk * 32, 16, 1024), idSS, kk > 0);
+            mma_ss(tmem + kColS, sdesc_at(kd, kk * 32), sdesc_at(qd, kk * 32), idSS, kk > 0);
           mma_commit(&S.s_full);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + kColDP, sdesc(v_addr + kk * 32, 16, 1024),
-                   sdesc(o_addr + kk * 32, 16, 1024), idSS, kk > 0);
+            mma_ss(tmem + kColDP, sdesc_at(vd, kk * 32), sdesc_at(od, kk * 32), idSS, kk > 0);
           mma_commit(&S.dp_full);
           return true;
         };
@@ -467,8 +468,9 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           if (u >= n_units) break;
           const int cnt = S.slot[sl].it.qend - S.slot[sl].it.qbeg;
           const int kb = n & 1;
-          k_addr = smem_u32(S.k[kb]);
-          v_addr = smem_u32(S.v[kb]);
+          kd = sdesc(smem_u32(S.k[kb]), 16, 1024);
+          vd = sdesc(smem_u32(S.v[kb]), 16, 1024);
+          kdm = sdesc(smem_u32(S.k[kb]), 16384, 1024);
           ok = mbar_wait(&S.kv_full[kb], (n >> 1) & 1, wait_ns, abort);
           // e = -1 issues S^T, dP^T of the unit's first tile; tile e issues
           // those of tile e + 1 as soon as the compute warps hold tile e's in
@@ -496,17 +498,18 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
               break;
             }
             tc_fence_after();
-            const uint32_t q_addr = smem_u32(S.q[s]), o_addr = smem_u32(S.dout[s]);
+            const uint64_t qdm = sdesc(smem_u32(S.q[s]), 16384, 1024);
+            const uint64_t odm = sdesc(smem_u32(S.dout[s]), 16384, 1024);
             // dV += P^T dO (P^T from TMEM), dK += dS^T Q: K = 128 queries in 8
             // steps of 16, the two accumulation chains interleaved
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t acc = (e > 0 || kk > 0) ? 1u : 0u;
-              mma_ts(tmem + kColDV, tmem + kColPT + kk * 8, sdesc(o_addr + kk * 2048, 16384, 1024),
+              mma_ts(tmem + kColDV, tmem + kColPT + kk * 8, sdesc_at(odm, kk * 2048),
                      idKM, acc);
               mma_ss(tmem + kColDK,
-                     sdesc(ds_addr + (kk >> 2) * kTileBytes + (kk & 3) * 32, 16, 1024),
-                     sdesc(q_addr + kk * 2048, 16384, 1024), idKM, acc);
+                     sdesc_at(dsk, (kk >> 2) * kTileBytes + (kk & 3) * 32),
+                     sdesc_at(qdm, kk * 2048), idKM, acc);
             }
             mma_commit(&S.empty[s]);  // Q, dO of this stage are no longer read
             if (gt > 0 && !mbar_wait(&S.dq_free, (gt - 1) & 1, wait_ns, abort)) {
@@ -517,8 +520,8 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             // dQ = dS K   (A = dS^T read MN-major, K = 128 keys)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tmem + kColDQ, sdesc(ds_addr + kk * 2048, kTileBytes, 1024),
-                     sdesc(k_addr + kk * 2048, 16384, 1024), idMM, kk > 0 ? 1u : 0u);
+              mma_ss(tmem + kColDQ, sdesc_at(dsm, kk * 2048), sdesc_at(kdm, kk * 2048), idMM,
+                     kk > 0 ? 1u : 0u);
             mma_commit(&S.dq_full);
             mma_commit(&S.pds_free);
           }

@@ -338,11 +338,11 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         const int s = g % NS;
         if (!mbar_wait(&S.k_full[s], (g / NS) & 1, wait_ns, abort)) return false;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(S.q[qb]), k_addr = smem_u32(S.k[s]);
+        const uint64_t qd = sdesc(smem_u32(S.q[qb]), 16, 1024);
+        const uint64_t kd = sdesc(smem_u32(S.k[s]), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + kColS, sdesc(q_addr + kk * 32, 16, 1024),
-                 sdesc(k_addr + kk * 32, 16, 1024), idS, kk > 0);
+          mma_ss(tmem + kColS, sdesc_at(qd, kk * 32), sdesc_at(kd, kk * 32), idS, kk > 0);
         mma_commit(&S.s_full);
         mma_commit(&S.k_empty[s]);
         return true;
@@ -420,10 +420,10 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
             break;
           }
           tc_fence_after();
-          const uint32_t v_addr = smem_u32(S.v[s]);
+          const uint64_t vd = sdesc(smem_u32(S.v[s]), 16384, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + kColO, tmem + kColP + kk * 8, sdesc(v_addr + kk * 2048, 16384, 1024),
+            mma_ts(tmem + kColO, tmem + kColP + kk * 8, sdesc_at(vd, kk * 2048),
                    idPV, (e > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&S.pv_done);
           mma_commit(&S.v_empty[s]);
@@ -506,23 +506,18 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           }
         }
       }
+      uint32_t w[32];
+#pragma unroll
+      for (int x = 0; x < 32; ++x) w[x] = pack2<F16>(o[2 * x], o[2 * x + 1]);
       // the row leaves in whole 32-byte sectors when the output allows it
       // (rows are 128 bytes, so all rows share the base's alignment)
       if ((reinterpret_cast<uintptr_t>(out) & 31) == 0) {
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t w[8];
-#pragma unroll
-          for (int x = 0; x < 8; ++x) w[x] = pack2<F16>(o[ch * 16 + 2 * x], o[ch * 16 + 2 * x + 1]);
-          st_global_v8(dst + 2 * ch, w);
-        }
+        for (int ch = 0; ch < 4; ++ch) st_global_v8(dst + 2 * ch, w + 8 * ch);
       } else {
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch)
-          dst[ch] = make_uint4(pack2<F16>(o[ch * 8 + 0], o[ch * 8 + 1]),
-                               pack2<F16>(o[ch * 8 + 2], o[ch * 8 + 3]),
-                               pack2<F16>(o[ch * 8 + 4], o[ch * 8 + 5]),
-                               pack2<F16>(o[ch * 8 + 6], o[ch * 8 + 7]));
+          dst[ch] = make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
       }
       lse[(size_t)pe.bh * g.T + pe.i] = L;
     };

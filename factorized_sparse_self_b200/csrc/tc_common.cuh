@@ -362,6 +362,13 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
   return d;
 }
 
+// The descriptor of the operand that starts `bytes` (a multiple of 16) past
+// the start of d's: the address field is (address >> 4) and shared-memory
+// addresses stay below 2^18, so the offset adds without a carry out of it.
+__device__ __forceinline__ uint64_t sdesc_at(uint64_t d, uint32_t bytes) {
+  return d + (bytes >> 4);
+}
+
 // Instruction descriptor of kind::f16 with 16-bit A and B (both fp16, or
 // both bf16) and an fp32 D: D format bits 4-5 (1 = f32), A format bits 7-9
 // and B format bits 10-12 (0 = f16, 1 = bf16), A / B major bits 15 / 16
