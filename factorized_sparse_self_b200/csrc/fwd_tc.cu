@@ -62,7 +62,10 @@ struct SmemFwd {
   uint64_t q_full[2], q_empty[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   uint64_t s_full, s_free, p_full, pv_done, o_free, fin;
   uint64_t sched_full[kSched], sched_empty[kSched];
-  int sched[kSched];  // work unit of each slot (n_units: no more work)
+  // published work units: index (n_units: no more work), head, item; the
+  // producer decodes each unit once and the other roles read it from here
+  int sched_u[kSched], sched_bh[kSched];
+  FwdItem sched_it[kSched];
   uint32_t tmem_base;
   int abort;
 };
@@ -203,10 +206,12 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
   };
   // Next published unit for a consuming role (one arrival per consuming warp).
   int sk = 0;
-  auto next_unit = [&](int& u, bool arrive) -> bool {
+  auto next_unit = [&](int& u, Unit& x, bool arrive) -> bool {
     const int k = sk % kSched;
     if (!mbar_wait(&S.sched_full[k], (sk / kSched) & 1, wait_ns, abort)) return false;
-    u = *reinterpret_cast<volatile int*>(&S.sched[k]);
+    u = *reinterpret_cast<volatile int*>(&S.sched_u[k]);
+    x.it = S.sched_it[k];
+    x.bh = S.sched_bh[k];
     if (arrive) mbar_arrive(&S.sched_empty[k]);
     ++sk;
     return true;
@@ -237,10 +242,14 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           u = (int)gridDim.x + atomicAdd(sched_slot, 1);
         }
       };
-      auto publish = [&](int u) -> bool {
+      auto publish = [&](int u, const Unit& y) -> bool {
         const int k = pub % kSched;
         if (!mbar_wait(&S.sched_empty[k], ((pub / kSched) & 1) ^ 1, wait_ns, abort)) return false;
-        S.sched[k] = u;
+        S.sched_u[k] = u;
+        if (u < n_units) {
+          S.sched_it[k] = y.it;
+          S.sched_bh[k] = y.bh;
+        }
         mbar_arrive(&S.sched_full[k]);
         ++pub;
         return true;
@@ -248,7 +257,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       Unit x;
       int cur = valid(blockIdx.x, x);
       while (ok && cur < n_units) {
-        if (!publish(cur)) {
+        if (!publish(cur, x)) {
           ok = false;
           break;
         }
@@ -281,7 +290,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         ++n;
         cur = valid(ticket, x);
       }
-      if (ok && !publish(n_units)) ok = false;  // no more work
+      if (ok && !publish(n_units, x)) ok = false;  // no more work
       if (!ok) fail();
       // no copy may be in flight when the CTA exits
       for (int b = 0; b < 2; ++b)
@@ -299,12 +308,12 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       bool ok = true;
       for (;;) {
         int u = 0;
-        if (!next_unit(u, true)) {
+        Unit x;
+        if (!next_unit(u, x, true)) {
           ok = false;
           break;
         }
         if (u >= n_units) break;
-        const Unit x = unit_of(items, u, NH, hs);
         for (int e = x.it.kbeg; e < x.it.kend; ++e, ++gt) {
           const int s = gt % NS;
           if (!mbar_wait(&S.v_empty[s], ((gt / NS) & 1) ^ 1, wait_ns, abort)) {
@@ -349,8 +358,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       };
       Unit cur, nx;
       int u = n_units, un = n_units;
-      ok = next_unit(u, true);
-      if (ok && u < n_units) cur = unit_of(items, u, NH, hs);
+      ok = next_unit(u, cur, true);
       bool first_done = false;  // S of this unit's first tile already issued ahead
       while (ok && u < n_units) {
         const int qb = n & 1;
@@ -377,12 +385,11 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           // by then all of this unit's K tiles have been issued, so the
           // producer has published it.
           if (e + 1 == cnt) {
-            if (!next_unit(un, true)) {
+            if (!next_unit(un, nx, true)) {
               ok = false;
               break;
             }
             have_next = true;
-            if (un < n_units) nx = unit_of(items, un, NH, hs);
           }
           // S of the next tile (this unit's, or the first of the next unit) goes
           // out as soon as the softmax has read S of this one, ahead of PV.
@@ -430,11 +437,10 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         }
         if (!ok) break;
         if (!have_next) {  // a unit without tiles
-          if (!next_unit(un, true)) {
+          if (!next_unit(un, nx, true)) {
             ok = false;
             break;
           }
-          if (un < n_units) nx = unit_of(items, un, NH, hs);
         }
         mma_commit(&S.q_empty[qb]);
         ++n;
@@ -528,7 +534,8 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
     };
     for (;;) {
       int u = 0;
-      const bool got = next_unit(u, false);
+      Unit x;
+      const bool got = next_unit(u, x, false);
       __syncwarp();
       if (lane == 0 && got) mbar_arrive(&S.sched_empty[(sk - 1) % kSched]);
       if (!__all_sync(0xffffffffu, got)) {
@@ -536,10 +543,10 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         break;
       }
       const bool end = u >= n_units;
-      Unit x;
-      x.it = FwdItem{0, 0, 0, 0, 0, 0, 0};
-      x.bh = 0;
-      if (!end) x = unit_of(items, u, NH, hs);
+      if (end) {
+        x.it = FwdItem{0, 0, 0, 0, 0, 0, 0};
+        x.bh = 0;
+      }
       const FwdItem& it = x.it;
       const int i = end ? -1 : view_pos(g, it.qview, it.qtile, row);
       const int iblk = i >= 0 ? fdiv(i, g.fl) : 0;
