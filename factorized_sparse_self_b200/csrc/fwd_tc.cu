@@ -9,9 +9,12 @@
 // Persistent CTAs, two per SM (96 KB shared memory and 256 TMEM columns
 // each, so the two CTAs of an SM interleave their MMA and softmax phases).
 // Work units (query tile x head, longest first) are claimed from a counter
-// by warp 4 and published to the other roles through a shared-memory ring,
-// so a CTA takes the next unit when it is ready for one. The counter is one
-// of the layout's slots; the last CTA to finish resets it. Warp roles:
+// by warp 4, decoded once (item and head) and published to the other roles
+// through a shared-memory ring, so a CTA takes the next unit when it is
+// ready for one. The counter is one of the layout's slots; the last CTA to
+// finish resets it. The second pass of a two-pass layout is a separate
+// instantiation (MERGE) that merges into the first pass's O and LSE; one-pass
+// launches carry no merge code. Warp roles:
 //   warp 4       TMA producer: claims the units; each unit's Q tile into one
 //                of two Q buffers (the next unit's Q loads while the current
 //                one computes) and K tiles into a 2-stage ring released by the
@@ -25,8 +28,9 @@
 //                row's live-key interval on PARTIAL tiles, keeps the running
 //                max (rescaling O in TMEM only when the max grows by more than
 //                2^8) and sum, writes P as bf16 pairs into TMEM; at the end of
-//                a unit normalises O, merges with a previous pass if asked,
-//                and stores O and LSE from registers.
+//                a unit normalises O, merges with the first pass (MERGE), and
+//                stores O (32-byte stores when the output allows) and LSE
+//                from registers.
 // Every wait is bounded; a wait that runs out sets the status word, raises
 // the CTA's abort flag, and all roles drain their in-flight work and return.
 #include <math.h>
