@@ -30,6 +30,9 @@ SMALL = [
     ("strided", "merged", 1, 2, 256, 64, 300, 1, "bf16", 0.5),   # l > T: full causal
     ("strided", "split", 1, 2, 384, 64, 384, 1, "bf16", 0.5),    # l = T: A2 is the diagonal
     ("fixed", "split", 1, 2, 256, 64, 300, 8, "bf16", 0.5),      # l > T
+    # divisors that are not powers of two in the kernels' index arithmetic:
+    ("strided", "merged", 1, 2, 3072, 64, 8, 1, "bf16", 0.5),    # 384-row classes, 3 tiles each
+    ("fixed", "merged", 3, 3, 1024, 64, 64, 8, "bf16", 0.5),     # 3 heads, 9 units per item
 ]
 
 
