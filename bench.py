@@ -78,6 +78,23 @@ def fwd_bytes(w):
     return rows * w.d * 2 * 4 + rows * 4
 
 
+def max_over_ranks(x, device):
+    """The largest of a float over all ranks (the slowest rank's time decides a
+    multi-GPU number); the value itself when there is one rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world, flops_per_rank, ms):
+    """Throughput of the whole job: every rank's work over the slowest time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def source_hash(path):
     with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
@@ -253,13 +270,9 @@ def run_ours(args):
         kb.append(st.st_kernel_elapsed_ms(1))
     st.st_kernel_timing(False)
     del graph
-    total_ms = sum(times)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(times), dev)
     ms_step = total_ms / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(world, flops, ms_step)
 
     # ---- end to end through the public API, host buffers ------------------------
     hq, hk, hv, hdo = (x.pin_memory() for x in (q, k, v, do))
@@ -314,12 +327,8 @@ def run_ours(args):
         et.append(e0.elapsed_time(e1))
     if st.st_last_device_status() != st.ST_OK:
         raise RuntimeError("device status error in the end-to-end steps")
-    e2e_ms = sum(et) / len(et)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(sum(et) / len(et), dev)
+    e2e_value = whole_job_tflops(world, flops, e2e_ms)
 
     # ---- roofline of the dominant kernel (the backward attention kernel) ------
     peaks, peak_src = load_peaks()
