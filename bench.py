@@ -78,6 +78,27 @@ def fwd_bytes(w):
     return rows * w.d * 2 * 4 + rows * 4
 
 
+def step_min_bytes(w):
+    """Fewest HBM bytes a fwd + bwd step can move: the forward reads Q, K, V and
+    writes O and LSE; the backward reads Q, K, V, O, dO and LSE and writes dQ,
+    dK, dV."""
+    rows = w.B * w.H * w.T
+    e = 2 if w.dtype == "bf16" else 4
+    return rows * w.d * e * 4 + rows * 4 + rows * w.d * e * 8 + rows * 4
+
+
+def step_roofline(w, flops, ms, peaks):
+    """The step's useful TFLOP/s against its roofline: the smaller of the
+    measured tensor peak and (useful flops / minimum bytes) x measured HBM
+    bandwidth."""
+    b = step_min_bytes(w)
+    roof = min(peaks["bf16_tflops"], flops / b * peaks["hbm_gbs"] * 1e9 / 1e12)
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"useful_tflops": achieved, "roofline_tflops": roof, "frac": achieved / roof,
+            "min_bytes": b, "flop_per_byte": flops / b,
+            "bound": "hbm" if roof < peaks["bf16_tflops"] else "tensor"}
+
+
 def max_over_ranks(x, device):
     """The largest of a float over all ranks (the slowest rank's time decides a
     multi-GPU number); the value itself when there is one rank."""
@@ -377,6 +398,10 @@ def run_ours(args):
         "ms_bwd_kernel": ms_b,
         "nnz": nnz,
         "useful_flops_per_step": flops,
+        # the same step counted without the backward's recomputation of S
+        "useful_flops_no_recompute_per_step": 12.0 * w.d * nnz,
+        "value_no_recompute": whole_job_tflops(world, 12.0 * w.d * nnz, ms_step),
+        "step_roofline": step_roofline(w, flops, ms_step, peaks),
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
@@ -438,9 +463,13 @@ def time_workload(st, w, steps=5, warmup=2, kind=None):
     assert st.st_last_device_status() == st.ST_OK
     nnz = nnz_of(L, w)
     ms = statistics.mean(tot)
+    peaks, _ = load_peaks()
+    flops = 14.0 * w.d * nnz
     return {"ms_step": ms, "ms_fwd_kernel": statistics.mean(tf),
             "ms_bwd_kernel": statistics.mean(tb), "nnz": nnz,
-            "useful_tflops": 14.0 * w.d * nnz / (ms * 1e-3) / 1e12,
+            "useful_tflops": flops / (ms * 1e-3) / 1e12,
+            "pct_of_peak": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "step_roofline": step_roofline(w, flops, ms, peaks),
             "fwd_tflops": 4.0 * w.d * nnz / (statistics.mean(tf) * 1e-3) / 1e12,
             "bwd_kernel_tflops": 10.0 * w.d * nnz / (statistics.mean(tb) * 1e-3) / 1e12}
 
