@@ -90,3 +90,30 @@ def test_invalid_descriptors_rejected():
         with pytest.raises(st.StatusError) as e:
             st.st_pattern_layout_host(*args)
         assert e.value.code == st.ST_ERR_INVALID
+
+
+def _golden_tiles():
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "layout_tiles.json")
+    with open(path) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _golden_tiles(),
+                         ids=lambda c: f"{c['kind']}-{c['mode']}-T{c['T']}-l{c['l']}-"
+                                       f"hc{c['head_class']}-seg{c['segment']}")
+def test_tile_coordinates_match_hand_derived_lists(orc, case):
+    """Pins the tile coordinates of the summary and residue-class orders: the
+    oracle's pair-by-pair tiling and the library's export must both give the
+    hand-derived (query tile, key tile, live) lists, not only the right totals."""
+    want = np.array(case["tiles"], dtype=np.int64)
+    args = (case["kind"], case["mode"], case["T"], case["l"], case["c"])
+    hc, seg = case["head_class"], case["segment"]
+    oq, ok, olive = orc.layout_tiles(*args, hc, seg)
+    np.testing.assert_array_equal(np.stack([oq, ok, olive], axis=1), want)
+    L = st.st_pattern_layout_host(*args)
+    ptr, idx, flags, live = L.export(hc, seg, transpose=False)
+    q, k, lv = _triples(ptr, idx, live, False)
+    np.testing.assert_array_equal(np.stack([q, k, lv], axis=1), want)
+    np.testing.assert_array_equal(flags, (want[:, 2] != 128 * 128).astype(np.uint8))
