@@ -7,11 +7,16 @@
 // a workspace between calls. For them this entry point uses a fixed scratch
 // array in the library's own device memory instead.
 //
-// The array is a file-scope __device__ variable, so every GPU that loads the
-// library holds it until the process exits. Host code cannot use its name as
-// a device address (in host code it is only a host-side stand-in), so the
-// device address is looked up with cudaGetSymbolAddress once per device, on
-// the first call made on that device, with that device current.
+// The array is a file-scope __device__ variable: it is created on a device
+// when the library's device code is loaded there and held until the process
+// exits. Under CUDA's default lazy loading that is the first call of this
+// entry point on the device (its cudaGetSymbolAddress); with
+// CUDA_MODULE_LOADING=EAGER it is when the process creates its context on
+// each device, whether or not this entry point is ever called. Host code
+// cannot use the array's name as a device address (in host code it is only a
+// host-side stand-in), so the device address is looked up with
+// cudaGetSymbolAddress once per device, on the first call made on that
+// device, with that device current.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -55,6 +60,11 @@ st_status st_sparse_attn_bwd_noalloc(const st_layout* layout, st_dtype dtype, in
   st_status s = st_sparse_attn_bwd_workspace(layout, dtype, B, H, T, d, &need);
   if (s != ST_OK) return s;
   if (need > kScratchBytes) return ST_ERR_WORKSPACE;
+  // the layout's device must be current before the array is looked up (and,
+  // under lazy loading, created) on it
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ST_ERR_CUDA;
+  if (!layout->on_device || dev != layout->device) return ST_ERR_INVALID;
   void* scratch = nullptr;
   s = scratch_address(&scratch);
   if (s != ST_OK) return s;

@@ -7,7 +7,11 @@
 //   dP^T = V dO^T
 //   P^T  = exp(scale S^T - LSE_i) on the live pairs, 0 elsewhere
 //   dS^T = P^T (dP^T - D_i),      D_i = dO_i . O_i (prologue kernel)
-//   dV  += P^T dO                 (M=128, N=64, K=128; P^T read from TMEM)
+//   dV  += P^T dO                 (M=128, N=64, K=128; P^T read from TMEM),
+//                                 in fp16: P^T rounded to fp16 and, for bf16
+//                                 inputs, dO copied to fp16 in place (times a
+//                                 power of two from the prologue's max |dO|)
+//                                 once dP^T has read it
 //   dK  += dS^T Q                 (dS^T from shared memory)
 //   dQ_i = dS K
 // dV and dK stay in TMEM for a whole work unit (a key tile, or a chunk of a
@@ -94,6 +98,7 @@ struct SmemBwd {
   uint64_t acc_full, acc_free, out_full, dst_free, kvst_free, fin;
   uint64_t sched_full[kSched], sched_empty[kSched];
   SchedSlot slot[kSched];        // published units
+  float bmax[8];                 // per compute warp: largest |dO| (start of the kernel)
   uint32_t tmem_base;
   int abort;
 };
@@ -220,7 +225,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
               float scale, float scale_log2, const float* __restrict__ lse,
               const float* __restrict__ Dg, ZeroRows zr, uint4* __restrict__ dq_out,
               uint4* __restrict__ dk_out, uint4* __restrict__ dv_out, int* sched_counter,
-              int* status, uint64_t wait_ns) {
+              const float* __restrict__ dmax_slots, int nslots, int* status, uint64_t wait_ns) {
   // The shared-memory plan fills the 227 KB a CTA may hold, with no room to
   // realign: the swizzled tiles need the dynamic window at a 1024-byte
   // boundary (where it starts when the kernel has no static shared memory).
@@ -424,11 +429,12 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       if (!ok && lane == 0) fail();
       if (lane == 0) {
         // the last K / V loads of both buffers have landed before the exit
+        // (these waits ignore the abort flag: the copies were issued and will land)
         for (int m = max(kv_last - 1, 0); m <= kv_last; ++m)
-          if (!mbar_wait(&S.kv_full[m & 1], (m >> 1) & 1, wait_ns, abort)) fail();
+          if (!mbar_wait_drain(&S.kv_full[m & 1], (m >> 1) & 1, wait_ns)) fail();
         for (int s = 0; s < NS; ++s)
           if (full_last[s] >= 0 &&
-              !mbar_wait(&S.full[s], (full_last[s] / NS) & 1, wait_ns, abort))
+              !mbar_wait_drain(&S.full[s], (full_last[s] / NS) & 1, wait_ns))
             fail();
       }
     } else if (warp == 9) {
@@ -436,6 +442,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       if (lane == 0) {
         const uint32_t idSS = idesc_16(128, 128, false, false, F16);
         const uint32_t idKM = idesc_16(128, 64, false, true, F16);  // A K-major, B MN-major
+        const uint32_t idDV = idesc_16(128, 64, false, true, true);  // fp16 P^T and dO
         const uint32_t idMM = idesc_16(128, 64, true, true, F16);   // A MN-major, B MN-major
         const uint32_t ds_addr = smem_u32(S.dst);
         const uint64_t dsk = sdesc(ds_addr, 16, 1024);          // dS^T, K-major (dK)
@@ -506,7 +513,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t acc = (e > 0 || kk > 0) ? 1u : 0u;
               mma_ts(tmem + kColDV, tmem + kColPT + kk * 8, sdesc_at(odm, kk * 2048),
-                     idKM, acc);
+                     idDV, acc);
               mma_ss(tmem + kColDK,
                      sdesc_at(dsk, (kk >> 2) * kTileBytes + (kk & 3) * 32),
                      sdesc_at(qdm, kk * 2048), idKM, acc);
@@ -532,8 +539,9 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           ++n;
         }
         if (!ok) fail();
+        // every MMA issued has completed before TMEM is freed
         mma_commit(&S.fin);
-        mbar_wait(&S.fin, 0, wait_ns, abort);
+        if (!mbar_wait_drain(&S.fin, 0, wait_ns)) fail();
       }
     } else if (warp == 10) {
       // ---------------- writer: TMA stores / reduce-adds of the staged tiles ----------------
@@ -658,6 +666,23 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
     const uint32_t st_addr = smem_u32(S.stage);
     int gt = 0, n = 0;
     int pend_direct = 0;  // q_direct of the tile whose dQ is pending
+    // dV is formed in fp16: for bf16 inputs dO is copied to fp16 times 2^e
+    // (e from the largest |dO|, over the prologue's per-block maxima), and the
+    // dV tile is scaled back by 2^-e when it is written
+    float do_scale = 1.f, dv_scale = 1.f;
+    if constexpr (!F16) {
+      float m = 0.f;
+      for (int x = threadIdx.x; x < nslots; x += 256) m = fmaxf(m, __ldg(dmax_slots + x));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      if (lane == 0) S.bmax[warp] = m;
+      named_sync(1, 256);
+#pragma unroll
+      for (int w2 = 0; w2 < 8; ++w2) m = fmaxf(m, S.bmax[w2]);
+      const int e = dout_exp(m);
+      do_scale = pow2f(e);
+      dv_scale = pow2f(-e);
+    }
 
     // dQ of tile t: TMEM -> registers -> staging (fp32 for the reduce-add, or
     // scaled bf16 for the direct store)
@@ -726,6 +751,26 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&S.sdp_free);  // S^T, dP^T of this tile may now be overwritten
+        if constexpr (!F16) {
+          // dP^T has read this stage's dO: turn it into the fp16 operand of dV
+          // (each thread converts 4 of the 1024 16-byte chunks; the swizzle
+          // moves whole chunks, so the element order inside them is kept)
+          const uint32_t da = smem_u32(S.dout[s]);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const uint32_t at = da + (uint32_t)(threadIdx.x + 256 * x) * 16u;
+            uint32_t w4[4];
+            ld_shared_v4(at, w4[0], w4[1], w4[2], w4[3]);
+#pragma unroll
+            for (int y = 0; y < 4; ++y) {
+              float lo, hi;
+              fmul2(lo, hi, __uint_as_float(w4[y] << 16), __uint_as_float(w4[y] & 0xffff0000u),
+                    do_scale, do_scale);
+              w4[y] = pack2<true>(lo, hi);
+            }
+            st_shared_v4(at, w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
         if (!full) mask_cols<2>(sv, wg * 64, lo, hi);
         const float* l2 = S.l2[s] + wg * 64;
         const float* dd = S.dd[s] + wg * 64;
@@ -750,7 +795,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
             float t0, t1, q0, q1;
             fadd2(t0, t1, dp[xk], dp[xk + 1], dv8[2 * x2], dv8[2 * x2 + 1]);
             fmul2(q0, q1, p0, p1, t0, t1);
-            pw[ch][x2] = pack2<F16>(p0, p1);
+            pw[ch][x2] = pack2<true>(p0, p1);
             dw[ch][x2] = pack2<F16>(q0, q1);
           }
         }
@@ -808,7 +853,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       const uint32_t dst =
           it.kv_direct ? kv_addr + (wg ? kTileBytes : 0) : (wg ? ds_addr : kv_addr);
       if (it.kv_direct) {
-        const float sc = wg ? 1.f : scale;  // dK carries the softmax scale, dV none
+        const float sc = wg ? dv_scale : scale;  // dK carries the softmax scale
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t o4[4];
@@ -846,7 +891,7 @@ template <bool F16>
 cudaError_t tc_bwd_t(const Call& c, const void* q, const void* k, const void* v,
                      const float* lse, const void* dout, const float* D, float* dq_acc,
                      float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv,
-                     int* sched_counter) {
+                     int* sched_counter, const float* slots, int nslots) {
   const st_layout* L = c.L;
   const int BH = c.B * c.H;
   if (L->dev.n_bwd_items == 0) return cudaSuccess;
@@ -899,8 +944,8 @@ cudaError_t tc_bwd_t(const Call& c, const void* q, const void* k, const void* v,
   bwd_tc_kernel<F16><<<grid, kThreads, smem, c.stream>>>(
       maps, L->geom, (const BwdItem*)L->dev.bwd_split[f], (int)units, NH,
       (const QEnt*)L->dev.q_ents, heads_of(c), c.scale, c.scale * kLog2e, lse, D,
-      zr, (uint4*)dq, (uint4*)dk, (uint4*)dv, sched_counter, c.status,
-      c.wait_ns);
+      zr, (uint4*)dq, (uint4*)dk, (uint4*)dv, sched_counter, slots, F16 ? 0 : nslots,
+      c.status, c.wait_ns);
   err = cudaGetLastError();
   record_end(c);
   return err;
@@ -910,11 +955,12 @@ cudaError_t tc_bwd_t(const Call& c, const void* q, const void* k, const void* v,
 
 cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v, const float* lse,
                    const void* dout, const float* D, float* dq_acc, float* dk_acc,
-                   float* dv_acc, void* dq, void* dk, void* dv, int* sched_counter) {
+                   float* dv_acc, void* dq, void* dk, void* dv, int* sched_counter,
+                   const float* slots, int nslots) {
   return c.dtype == ST_F16 ? tc_bwd_t<true>(c, q, k, v, lse, dout, D, dq_acc, dk_acc, dv_acc,
-                                            dq, dk, dv, sched_counter)
+                                            dq, dk, dv, sched_counter, slots, nslots)
                            : tc_bwd_t<false>(c, q, k, v, lse, dout, D, dq_acc, dk_acc, dv_acc,
-                                             dq, dk, dv, sched_counter);
+                                             dq, dk, dv, sched_counter, slots, nslots);
 }
 
 }  // namespace st

@@ -315,7 +315,7 @@ st_status st_sparse_attn_bwd_workspace(const st_layout* L, st_dtype dtype, int32
   if (dtype != ST_F32 && dtype != ST_BF16 && dtype != ST_F16) return ST_ERR_INVALID;
   const size_t rows = (size_t)B * H * T;
   size_t b = round256(rows * sizeof(float));  // D
-  if (dtype != ST_F32) b += 3 * round256(rows * (size_t)d * sizeof(float)) + 256;
+  if (dtype != ST_F32) b += 3 * round256(rows * (size_t)d * sizeof(float)) + kMiscBytes;
   *bytes = b;
   return ST_OK;
 }
@@ -369,12 +369,15 @@ st_status st_sparse_attn_bwd_heads(const st_layout* L, st_dtype dtype, int32_t B
     float* dk_acc = acc + stride;
     float* dv_acc = acc + 2 * stride;
     int* counter = reinterpret_cast<int*>(dv_acc + stride);  // work counter of the kernel
-    e = bwd_prep(c, o, dout, Dv, dq_acc, dk_acc, dv_acc, counter);
+    float* slots = reinterpret_cast<float*>(reinterpret_cast<char*>(counter) + 256);
+    int nslots = 0;
+    e = bwd_prep(c, o, dout, Dv, dq_acc, dk_acc, dv_acc, counter, slots, &nslots);
     Call cm = c;
     arm(cm, 1);
     if (e == cudaSuccess)
-      e = tc_bwd(cm, q, k, v, lse, dout, Dv, dq_acc, dk_acc, dv_acc, dq, dk, dv, counter);
-    if (e == cudaSuccess) e = bwd_finish(c, dq_acc, dk_acc, dv_acc, dq, dk, dv);
+      e = tc_bwd(cm, q, k, v, lse, dout, Dv, dq_acc, dk_acc, dv_acc, dq, dk, dv, counter, slots,
+                 nslots);
+    if (e == cudaSuccess) e = bwd_finish(c, dq_acc, dk_acc, dv_acc, slots, nslots, dq, dk, dv);
   }
   return e == cudaSuccess ? ST_OK : ST_ERR_CUDA;
 }

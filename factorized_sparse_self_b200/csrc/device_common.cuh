@@ -84,6 +84,19 @@ __device__ __forceinline__ int class_of(int bh, const Heads& hs) {
   return hs.nclasses == 2 ? ((bh % hs.H) & 1) : 0;
 }
 
+// The backward pass of the 16-bit path forms dV from P and dout rounded to
+// fp16 (three more significant bits for P than bf16 gives). dout enters that
+// product as dout * 2^e, with e chosen from m = max |dout| so that
+// m * 2^e lies in [2^13, 2^14): far from fp16 overflow, and every bf16 value
+// within 2^27 of m keeps all its bits. e = 0 for m = 0 (or not finite).
+__device__ __forceinline__ int dout_exp(float m) {
+  if (!(m > 0.f) || !(m < INFINITY)) return 0;
+  const int E = (int)((__float_as_uint(m) >> 23) & 0xffu);  // m in [2^(E-127), 2^(E-126))
+  return max(-100, min(100, 140 - E));
+}
+// 2^e for -126 <= e <= 127.
+__device__ __forceinline__ float pow2f(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
+
 __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }

@@ -296,12 +296,13 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       }
       if (ok && !publish(n_units, x)) ok = false;  // no more work
       if (!ok) fail();
-      // no copy may be in flight when the CTA exits
+      // no copy may be in flight when the CTA exits (these waits ignore the
+      // abort flag: the copies were issued and will land)
       for (int b = 0; b < 2; ++b)
-        if (q_last[b] >= 0 && !mbar_wait(&S.q_full[b], (q_last[b] >> 1) & 1, wait_ns, abort))
+        if (q_last[b] >= 0 && !mbar_wait_drain(&S.q_full[b], (q_last[b] >> 1) & 1, wait_ns))
           fail();
       for (int s = 0; s < NS; ++s)
-        if (kv_last[s] >= 0 && !mbar_wait(&S.k_full[s], (kv_last[s] / NS) & 1, wait_ns, abort))
+        if (kv_last[s] >= 0 && !mbar_wait_drain(&S.k_full[s], (kv_last[s] / NS) & 1, wait_ns))
           fail();
     }
   } else if (warp == 6) {
@@ -336,7 +337,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
       }
       if (!ok) fail();
       for (int s = 0; s < NS; ++s)
-        if (v_last[s] >= 0 && !mbar_wait(&S.v_full[s], (v_last[s] / NS) & 1, wait_ns, abort))
+        if (v_last[s] >= 0 && !mbar_wait_drain(&S.v_full[s], (v_last[s] / NS) & 1, wait_ns))
           fail();
     }
   } else if (warp == 5) {
@@ -452,8 +453,9 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
         cur = nx;
       }
       if (!ok) fail();
+      // every MMA issued has completed before TMEM is freed
       mma_commit(&S.fin);
-      mbar_wait(&S.fin, 0, wait_ns, abort);
+      if (!mbar_wait_drain(&S.fin, 0, wait_ns)) fail();
     }
   }
   } else {

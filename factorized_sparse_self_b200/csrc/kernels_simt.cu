@@ -318,63 +318,92 @@ __device__ __forceinline__ float dot8(const uint4& a, const uint4& b) {
   return s;
 }
 
+// Largest |x| of eight bf16 values, as a bf16 bit pattern (the magnitude
+// bits of a bf16 order like the values for every non-NaN input).
+__device__ __forceinline__ uint32_t absmax8_bf16(const uint4& a) {
+  const uint32_t m = 0x7fff7fffu;
+  const uint32_t x = __vmaxu2(__vmaxu2(a.x & m, a.y & m), __vmaxu2(a.z & m, a.w & m));
+  return max(x & 0xffffu, x >> 16);
+}
+
+// Backward prologue of the 16-bit path. Grid (bx, gy): blockIdx.x strides over
+// the rows of one head, blockIdx.y over the selected heads of every batch
+// entry (gy <= kDoutSlots / bx). Writes D_i = dout_i . O_i for every row,
+// zeroes the fp32 accumulator rows that collect several contributions and
+// the backward kernel's work counter, and (bf16) the largest |dout| seen by
+// each block into slots[blockIdx.y * gridDim.x + blockIdx.x], from which the
+// backward kernel takes the power-of-two scale of its fp16 copy of dout.
 template <bool F16>
 __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
                                 float* __restrict__ Dv,
                                 int T, Heads hs, RowSet rs, float4* __restrict__ dq_acc,
                                 float4* __restrict__ dk_acc, float4* __restrict__ dv_acc,
-                                int* __restrict__ sched_counter) {
-  // grid.y runs over the selected heads of every batch
-  const int bh = (blockIdx.y / hs.hn) * hs.H + hs.h0 + blockIdx.y % hs.hn;
+                                int* __restrict__ sched_counter, float* __restrict__ slots) {
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *sched_counter = 0;
-  const int hc = class_of(bh, hs);
-  const size_t rb = (size_t)bh * T;
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int stride = gridDim.x * blockDim.x;
-  // D: eight lanes per 128-byte row (one 16-byte chunk each), four rows per
-  // warp and pass, four passes' loads in flight per thread
-  {
-    const int lane = threadIdx.x & 31, sub = lane & 7;
-    const int rstep = stride >> 3;  // rows per pass over the grid (multiple of 4)
-    const uint4* o4 = o + rb * 8;
-    const uint4* d4 = dout + rb * 8;
-    for (int rw = (tid >> 5) * 4; rw < T; rw += 4 * rstep) {  // warp-uniform
-      uint4 a[4], b[4];
+  const int lane = threadIdx.x & 31, sub = lane & 7;
+  const int nheads = hs.B * hs.hn;
+  uint32_t amax = 0;  // bf16 bits of the largest |dout| this thread read
+  for (int y = blockIdx.y; y < nheads; y += gridDim.y) {
+    const int bh = (y / hs.hn) * hs.H + hs.h0 + y % hs.hn;
+    const int hc = class_of(bh, hs);
+    const size_t rb = (size_t)bh * T;
+    // D: eight lanes per 128-byte row (one 16-byte chunk each), four rows per
+    // warp and pass, four passes' loads in flight per thread
+    {
+      const int rstep = stride >> 3;  // rows per pass over the grid (multiple of 4)
+      const uint4* o4 = o + rb * 8;
+      const uint4* d4 = dout + rb * 8;
+      for (int rw = (tid >> 5) * 4; rw < T; rw += 4 * rstep) {  // warp-uniform
+        uint4 a[4], b[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = rw + (lane >> 3) + u * rstep;
-        a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
-        if (r < T) {
-          a[u] = __ldg(o4 + (size_t)r * 8 + sub);
-          b[u] = __ldg(d4 + (size_t)r * 8 + sub);
+        for (int u = 0; u < 4; ++u) {
+          const int r = rw + (lane >> 3) + u * rstep;
+          a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (r < T) {
+            a[u] = __ldg(o4 + (size_t)r * 8 + sub);
+            b[u] = __ldg(d4 + (size_t)r * 8 + sub);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if constexpr (!F16) amax = max(amax, absmax8_bf16(b[u]));
+          float sacc = dot8<F16>(a[u], b[u]);
+          sacc += __shfl_xor_sync(0xffffffffu, sacc, 4);
+          sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
+          sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
+          const int r = rw + (lane >> 3) + u * rstep;
+          if (sub == 0 && r < T) Dv[rb + r] = sacc;
         }
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        float sacc = dot8<F16>(a[u], b[u]);
-        sacc += __shfl_xor_sync(0xffffffffu, sacc, 4);
-        sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
-        sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
-        const int r = rw + (lane >> 3) + u * rstep;
-        if (sub == 0 && r < T) Dv[rb + r] = sacc;
+    }
+    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    {
+      int nr;
+      const int32_t* rows = rows_of(rs, hc, ROWS_Q_ACC, nr);
+      for (int64_t x = tid; x < (int64_t)nr * 16; x += stride)
+        dq_acc[(rb + rows[x >> 4]) * 16 + (x & 15)] = z4;
+    }
+    {
+      int nr;
+      const int32_t* rows = rows_of(rs, hc, ROWS_K_ACC, nr);
+      for (int64_t x = tid; x < (int64_t)nr * 16; x += stride) {
+        const size_t e = (rb + rows[x >> 4]) * 16 + (x & 15);
+        dk_acc[e] = z4;
+        dv_acc[e] = z4;
       }
     }
   }
-  const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-  {
-    int nr;
-    const int32_t* rows = rows_of(rs, hc, ROWS_Q_ACC, nr);
-    for (int64_t x = tid; x < (int64_t)nr * 16; x += stride)
-      dq_acc[(rb + rows[x >> 4]) * 16 + (x & 15)] = z4;
-  }
-  {
-    int nr;
-    const int32_t* rows = rows_of(rs, hc, ROWS_K_ACC, nr);
-    for (int64_t x = tid; x < (int64_t)nr * 16; x += stride) {
-      const size_t e = (rb + rows[x >> 4]) * 16 + (x & 15);
-      dk_acc[e] = z4;
-      dv_acc[e] = z4;
-    }
+  // the block's largest |dout|: warp, then block (bf16 bits widen to fp32 bits)
+  __shared__ uint32_t wmax[32];
+  amax = __reduce_max_sync(0xffffffffu, amax);
+  if (lane == 0) wmax[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t m = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = max(m, wmax[w]);
+    slots[blockIdx.y * gridDim.x + blockIdx.x] = __uint_as_float(m << 16);
   }
 }
 
@@ -396,13 +425,24 @@ __device__ __forceinline__ uint4 round8f(const float4& a, const float4& b, float
 }
 
 // Rounds the accumulated rows: eight elements (two float4 in, 16 bytes out)
-// per thread and step.
+// per thread and step. dV partials carry the factor 2^e of the backward's
+// fp16 dout (from the prologue's slots; nslots = 0 means e = 0).
 template <bool F16>
 __global__ void bwd_finish_kernel(const float4* __restrict__ dq_acc,
                                   const float4* __restrict__ dk_acc,
                                   const float4* __restrict__ dv_acc, int T, Heads hs,
-                                  RowSet rs, float scale, uint4* __restrict__ dq,
+                                  RowSet rs, float scale, const float* __restrict__ slots,
+                                  int nslots, uint4* __restrict__ dq,
                                   uint4* __restrict__ dk, uint4* __restrict__ dv) {
+  __shared__ float bmax[32];
+  float m = 0.f;
+  for (int s = threadIdx.x; s < nslots; s += blockDim.x) m = fmaxf(m, __ldg(slots + s));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) bmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, bmax[w]);
+  const float dv_scale = pow2f(-dout_exp(m));
   const int bh = (blockIdx.y / hs.hn) * hs.H + hs.h0 + blockIdx.y % hs.hn;
   const int hc = class_of(bh, hs);
   const size_t rb = (size_t)bh * T;
@@ -422,7 +462,7 @@ __global__ void bwd_finish_kernel(const float4* __restrict__ dq_acc,
     for (int64_t x = tid; x < (int64_t)nr * 8; x += stride) {
       const size_t e = (rb + rows[x >> 3]) * 8 + (x & 7);
       dk[e] = round8f<F16>(__ldg(dk_acc + 2 * e), __ldg(dk_acc + 2 * e + 1), scale);
-      dv[e] = round8f<F16>(__ldg(dv_acc + 2 * e), __ldg(dv_acc + 2 * e + 1), 1.f);
+      dv[e] = round8f<F16>(__ldg(dv_acc + 2 * e), __ldg(dv_acc + 2 * e + 1), dv_scale);
     }
   }
 }
@@ -531,20 +571,29 @@ cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* 
   return cudaGetLastError();
 }
 
-cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* Dv, float* dq_acc,
-                     float* dk_acc, float* dv_acc, int* sched_counter) {
+int prep_grid(const Call& c, dim3& grid) {
   const int T = c.L->geom.T;
   const int bx = std::max(1, std::min(64, (T + 127) / 128));
-  dim3 grid(bx, c.B * c.hn);
+  const int gy = std::max(1, std::min(c.B * c.hn, kDoutSlots / bx));
+  grid = dim3(bx, gy);
+  return bx * gy;
+}
+
+cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* Dv, float* dq_acc,
+                     float* dk_acc, float* dv_acc, int* sched_counter, float* slots,
+                     int* nslots) {
+  dim3 grid;
+  *nslots = prep_grid(c, grid);
   auto kern = (c.dtype == ST_F16) ? bwd_prep_kernel<true> : bwd_prep_kernel<false>;
   kern<<<grid, 256, 0, c.stream>>>(
-      (const uint4*)o, (const uint4*)dout, Dv, T, heads_of(c),
-      row_set_of(c.L), (float4*)dq_acc, (float4*)dk_acc, (float4*)dv_acc, sched_counter);
+      (const uint4*)o, (const uint4*)dout, Dv, c.L->geom.T, heads_of(c),
+      row_set_of(c.L), (float4*)dq_acc, (float4*)dk_acc, (float4*)dv_acc, sched_counter, slots);
   return cudaGetLastError();
 }
 
 cudaError_t bwd_finish(const Call& c, const float* dq_acc, const float* dk_acc,
-                       const float* dv_acc, void* dq, void* dk, void* dv) {
+                       const float* dv_acc, const float* slots, int nslots, void* dq, void* dk,
+                       void* dv) {
   const st_layout* L = c.L;
   int most = 0;
   for (int hc = 0; hc < (int)L->hcs.size(); ++hc)
@@ -555,7 +604,8 @@ cudaError_t bwd_finish(const Call& c, const float* dq_acc, const float* dk_acc,
   auto kern = (c.dtype == ST_F16) ? bwd_finish_kernel<true> : bwd_finish_kernel<false>;
   kern<<<grid, 256, 0, c.stream>>>(
       (const float4*)dq_acc, (const float4*)dk_acc, (const float4*)dv_acc, L->geom.T,
-      heads_of(c), row_set_of(L), c.scale, (uint4*)dq, (uint4*)dk, (uint4*)dv);
+      heads_of(c), row_set_of(L), c.scale, slots, c.dtype == ST_F16 ? 0 : nslots, (uint4*)dq,
+      (uint4*)dk, (uint4*)dv);
   return cudaGetLastError();
 }
 

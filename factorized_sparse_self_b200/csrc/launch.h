@@ -46,15 +46,19 @@ cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* 
                          size_t acc_elems);
 
 // 16-bit backward, around the tensor-core kernel: bwd_prep writes D for every
-// row and zeroes the fp32 accumulator rows that collect several contributions
-// and the work counter the tensor-core kernel claims its units from;
+// row, zeroes the fp32 accumulator rows that collect several contributions
+// and the work counter the tensor-core kernel claims its units from, and
+// writes the largest |dout| of each of its *nslots blocks into slots;
 // bwd_finish rounds the accumulated rows into dq, dk, dv (scale applied to dQ
-// and dK). Rows that a single backward unit produces, and rows nobody writes
-// (zero-filled), are written by the tensor-core kernel itself.
+// and dK, the inverse of the dout scale to dV). Rows that a single backward
+// unit produces, and rows nobody writes (zero-filled), are written by the
+// tensor-core kernel itself.
 cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* D, float* dq_acc,
-                     float* dk_acc, float* dv_acc, int* sched_counter);
+                     float* dk_acc, float* dv_acc, int* sched_counter, float* slots,
+                     int* nslots);
 cudaError_t bwd_finish(const Call& c, const float* dq_acc, const float* dk_acc,
-                       const float* dv_acc, void* dq, void* dk, void* dv);
+                       const float* dv_acc, const float* slots, int nslots, void* dq, void* dk,
+                       void* dv);
 
 // Tensor-core path (tcgen05 + TMA): bf16, d = 64.
 cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, void* o,
@@ -62,7 +66,7 @@ cudaError_t tc_fwd(const Call& c, const void* q, const void* k, const void* v, v
 cudaError_t tc_bwd(const Call& c, const void* q, const void* k, const void* v,
                    const float* lse, const void* dout, const float* D, float* dq_acc,
                    float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv,
-                   int* sched_counter);
+                   int* sched_counter, const float* slots, int nslots);
 
 }  // namespace st
 

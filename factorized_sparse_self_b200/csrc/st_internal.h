@@ -13,6 +13,12 @@ namespace st {
 constexpr int kTile = 128;  // query and key tile edge, in view rows
 constexpr int kBwdChunk = 8; // most query tiles one backward work item visits
 constexpr int kSchedSlots = 64;  // forward calls of one layout that may run at once
+// Blocks of the 16-bit backward prologue, each reporting its largest |dout|
+// (the backward kernel scales its fp16 copy of dout by a power of two).
+constexpr int kDoutSlots = 1024;
+// Tail of the 16-bit backward workspace: the backward kernel's work counter
+// (first 256 bytes), then kDoutSlots floats.
+constexpr size_t kMiscBytes = 256 + 4 * kDoutSlots;
 
 // Row orders ("views") a segment reads its queries or keys in.
 enum View : uint8_t {

@@ -83,6 +83,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Waits for a phase that work this CTA has already issued will complete (its
+// own TMA copies or MMAs): gives up only after limit_ns, never on the abort
+// flag, so that no CTA exits, or frees TMEM, with such work still in flight.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
+                                                uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > limit_ns) return false;
+  }
+}
+
 // ---- packed fp32 arithmetic and 3-input max (sm_100) ---------------------------
 
 // (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1), one fma.rn.f32x2.

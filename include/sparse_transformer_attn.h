@@ -186,11 +186,15 @@ st_status st_sparse_attn_bwd_heads(const st_layout* layout, st_dtype dtype, int3
  * latency-critical path that must not allocate). This entry point computes
  * exactly what st_sparse_attn_bwd computes, with the same arguments except
  * the workspace: its scratch is a fixed 64 MiB array of library-owned device
- * memory that every GPU which loads the library holds until the process
- * exits. It never allocates.
+ * memory, held until the process exits by every GPU where the library's
+ * device code is loaded: under CUDA's default lazy module loading, a GPU on
+ * which this entry point has been called; with CUDA_MODULE_LOADING=EAGER,
+ * every GPU on which the process creates a context. It never allocates.
  *  - Limit: st_sparse_attn_bwd_workspace bytes for these sizes must not
- *    exceed 64 MiB (bf16: B*H*T*(4 + 12*d) + 256 bytes, rounded up); larger
- *    calls return ST_ERR_WORKSPACE before any launch.
+ *    exceed 64 MiB (bf16: B*H*T*(4 + 12*d) + 4352 bytes, each part rounded
+ *    up to 256 bytes); larger calls return ST_ERR_WORKSPACE before any
+ *    launch. A layout built on another device than the current one returns
+ *    ST_ERR_INVALID before the array is touched.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.
@@ -205,8 +209,10 @@ st_status st_sparse_attn_bwd_noalloc(const st_layout* layout, st_dtype dtype, in
                                      void* dv, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device-side status word
- * that the kernels set when a bounded wait runs out (ST_ERR_DEVICE_TIMEOUT) or
- * an index check fails (ST_ERR_INVALID); ST_ERR_CUDA if the sync fails. */
+ * of the current device: ST_ERR_DEVICE_TIMEOUT after a kernel's bounded wait
+ * ran out, ST_ERR_UNSUPPORTED if the backward kernel found its shared memory
+ * misaligned (it then computes nothing); ST_OK otherwise. ST_ERR_CUDA if the
+ * sync fails. */
 st_status st_last_device_status(void* stream);
 
 /* Upper bound, in nanoseconds, of every on-device wait of later launches

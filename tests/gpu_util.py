@@ -53,8 +53,9 @@ def device_inputs(B, H, T, d, dtype, std, seed=0):
     return (q, k, v, do), tuple(x.cuda() for x in (q, k, v, do))
 
 
-def run_library(layout, qd, kd, vd, dod, backward=True):
-    o, lse = st.st_sparse_attn_fwd(layout, qd, kd, vd)
+def run_library(layout, qd, kd, vd, dod, backward=True, forward=None):
+    """Forward (or the given (o, lse)) and backward through the C ABI."""
+    o, lse = forward if forward is not None else st.st_sparse_attn_fwd(layout, qd, kd, vd)
     grads = None
     if backward:
         grads = st.st_sparse_attn_bwd(layout, qd, kd, vd, o, lse, dod)

@@ -33,6 +33,11 @@ SMALL = [
     # divisors that are not powers of two in the kernels' index arithmetic:
     ("strided", "merged", 1, 2, 3072, 64, 8, 1, "bf16", 0.5),    # 384-row classes, 3 tiles each
     ("fixed", "merged", 3, 3, 1024, 64, 64, 8, "bf16", 0.5),     # 3 heads, 9 units per item
+    # 18 heads of the fixed split pattern at std 0.5: the first key of a block
+    # collects up to l query rows with large weights (max |dV| about 6); with P
+    # rounded to bf16 before the dV product this case measured dV max-abs
+    # 0.0213, so it pins the fp16 P^T / dO operands of that product
+    ("fixed", "split", 3, 6, 1024, 64, 64, 8, "bf16", 0.5),
 ]
 
 
@@ -53,33 +58,44 @@ def test_parity_small(orc, case):
 
 
 @pytest.mark.parametrize("name", [n for n in synth.ORDER if synth.WORKLOADS[n].dtype == "bf16"])
-def test_parity_full_size_sampled(orc, name):
-    """Full workload sizes, launched as the benchmark launches them: sampled
-    output rows vs the oracle row by row (forward rows, dQ rows, dK / dV rows)."""
+def test_parity_full_size(orc, name):
+    """Full workload sizes, launched as the benchmark launches them: every
+    element of O, LSE, dQ, dK and dV against the oracle on the same inputs."""
     w = synth.WORKLOADS[name]
     (q, k, v, do), (qd, kd, vd, dod) = device_inputs(w.B, w.H, w.T, w.d, w.dtype, w.std, seed=0)
     L = st.st_pattern_layout(w.kind, w.mode, w.T, w.l, w.c)
     o, lse, (dq, dk, dv) = run_library(L, qd, kd, vd, dod)
-    rng = np.random.default_rng(1)
-    BH = w.B * w.H
-    n = 24
-    bh = rng.integers(0, BH, n)
-    rows = np.concatenate([rng.integers(0, w.T, n - 4), [0, w.T - 1, w.l - 1, w.l]])
-    # include the last summary key of block 0 and the first row of block 1
     qf, kf, vf, dof = f32(q), f32(k), f32(v), f32(do)
-    ro, rlse = orc.forward_rows(w.kind, w.mode, qf, kf, vf, w.l, w.c, bh, rows)
-    go = f32(o.cpu()).reshape(BH, w.T, w.d)[bh, rows]
-    compare("O rows", go, ro, "bf16", name)
-    compare_lse(lse.cpu().numpy().reshape(BH, w.T)[bh, rows], rlse, "bf16", name)
-    rdq = orc.backward_query_rows(w.kind, w.mode, qf, kf, vf, dof, w.l, w.c, bh, rows)
-    compare("dQ rows", f32(dq.cpu()).reshape(BH, w.T, w.d)[bh, rows], rdq, "bf16", name)
-    nk = 6
-    kb, kr = bh[:nk], rows[:nk].copy()
-    if w.kind == "fixed":
-        kr[0] = w.l - 1  # a summary key, attended by every later block
-    rdk, rdv = orc.backward_key_rows(w.kind, w.mode, qf, kf, vf, dof, w.l, w.c, kb, kr)
-    compare("dK rows", f32(dk.cpu()).reshape(BH, w.T, w.d)[kb, kr], rdk, "bf16", name)
-    compare("dV rows", f32(dv.cpu()).reshape(BH, w.T, w.d)[kb, kr], rdv, "bf16", name)
+    del q, k, v, do
+    ro, rlse = orc.forward(w.kind, w.mode, qf, kf, vf, w.l, w.c)
+    compare("O", f32(o.cpu()), ro, "bf16", name)
+    compare_lse(lse.cpu().numpy(), rlse, "bf16", name)
+    del ro, rlse
+    rdq, rdk, rdv = orc.backward(w.kind, w.mode, qf, kf, vf, dof, w.l, w.c)
+    compare("dQ", f32(dq.cpu()), rdq, "bf16", name)
+    compare("dK", f32(dk.cpu()), rdk, "bf16", name)
+    compare("dV", f32(dv.cpu()), rdv, "bf16", name)
+
+
+def test_backward_run_to_run_drift_is_bounded():
+    """The backward sums partial dQ (and, for long key columns, dK / dV) tiles
+    with fp32 reduce-adds in L2, whose order varies between runs; it is not
+    bitwise reproducible. Rows with a single writer are; an accumulated value
+    x = sum of k partials may move by the fp32 summation order, at most about
+    k * 2^-24 times the partials' magnitude (bounded here by 2^-16 of the
+    tensor's largest entry), and then by one bf16 rounding step on each run
+    (2^-8 of |x| each)."""
+    w = synth.WORKLOADS["fixed-merged-T12288"]
+    (_, _, _, _), (qd, kd, vd, dod) = device_inputs(w.B, w.H, w.T, w.d, w.dtype, w.std)
+    L = st.st_pattern_layout(w.kind, w.mode, w.T, w.l, w.c)
+    o, lse, g1 = run_library(L, qd, kd, vd, dod)
+    g1 = [x.clone() for x in g1]
+    _, _, g2 = run_library(L, qd, kd, vd, dod, forward=(o, lse))
+    for name, a, b in zip(("dQ", "dK", "dV"), g1, g2):
+        a, b = a.float(), b.float()
+        bound = torch.maximum(a.abs(), b.abs()) * 2.0 ** -7 + a.abs().max() * 2.0 ** -16
+        excess = ((a - b).abs() - bound).max().item()
+        assert excess <= 0, f"{name}: run-to-run difference exceeds its bound by {excess:.3g}"
 
 
 def test_full_size_invariants():
