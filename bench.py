@@ -31,7 +31,7 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-HEADLINE = "fixed-split-T4096"
+HEADLINE = "fixed-merged-T12288"
 METRIC = "sparse attn fwd+bwd useful TFLOP/s and % of B200 bf16 tensor-core peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
@@ -97,6 +97,40 @@ def step_roofline(w, flops, ms, peaks):
     return {"useful_tflops": achieved, "roofline_tflops": roof, "frac": achieved / roof,
             "min_bytes": b, "flop_per_byte": flops / b,
             "bound": "hbm" if roof < peaks["bf16_tflops"] else "tensor"}
+
+
+def kernel_roofline(w, nnz, ms_bwd, peaks, peak_src):
+    """Roofline of the dominant kernel (the backward attention kernel): its
+    algorithmic bytes or flops per launch over its CUDA-event duration, against
+    the measured peak of the resource that bounds it (HBM below the ridge,
+    the bf16 tensor pipe above)."""
+    bwd_flops = 10.0 * w.d * nnz
+    bwd_b = bwd_bytes(w)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if bwd_flops / bwd_b < ridge:
+        achieved = bwd_b / (ms_bwd * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = bwd_flops / (ms_bwd * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = recorded_traffic("bwd_tc.cu", w.name)
+    roof["kernel"] = "bwd_tc_kernel"
+    roof["peak_source"] = f"{peak_src} (burst)"
+    roof["algorithmic_bytes"] = bwd_b
+    roof["algorithmic_flops"] = bwd_flops
+    roof["ms_per_launch"] = ms_bwd
+    return roof
+
+
+def workload_config(w, world):
+    """The `config` object of a bench line (both arms use the same one)."""
+    return {"workload": w.name, "pattern": w.kind, "heads": w.mode, "B_per_gpu": w.B,
+            "global_batch": w.B * world, "H": w.H, "T": w.T, "d": w.d, "l": w.l, "c": w.c,
+            "parallelism": f"dp{world} (independent heads per GPU)",
+            "l2": "flushed between timed steps (256 MB write)",
+            "launch": "timed step = one CUDA-graph replay of the fwd + bwd calls"}
 
 
 def max_over_ranks(x, device):
@@ -355,23 +389,7 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     ms_f = statistics.mean(kf)
     ms_b = statistics.mean(kb)
-    bwd_flops = 10.0 * w.d * nnz
-    bwd_b = bwd_bytes(w)
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if bwd_flops / bwd_b < ridge:
-        achieved = bwd_b / (ms_b * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-    else:
-        achieved = bwd_flops / (ms_b * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = recorded_traffic("bwd_tc.cu", w.name)
-    roof["kernel"] = "bwd_tc_kernel"
-    roof["peak_source"] = f"{peak_src} (burst)"
-    roof["algorithmic_bytes"] = bwd_b
-    roof["algorithmic_flops"] = bwd_flops
-    roof["ms_per_launch"] = ms_b
+    roof = kernel_roofline(w, nnz, ms_b, peaks, peak_src)
 
     fl, bl = L.launches(dt_code)
     line = {
@@ -387,11 +405,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded N(0, std) Q, K, V; N(0,1) dO)",
-        "config": {"workload": w.name, "pattern": w.kind, "heads": w.mode, "B_per_gpu": w.B,
-                   "global_batch": w.B * world, "H": w.H, "T": w.T, "d": w.d, "l": w.l,
-                   "c": w.c, "parallelism": f"dp{world} (independent heads per GPU)",
-                   "l2": "flushed between timed steps (256 MB write)",
-                   "launch": "timed step = one CUDA-graph replay of the fwd + bwd calls"},
+        "config": workload_config(w, world),
         "pct_of_peak": value / peaks["bf16_tflops"],
         "pct_of_spec_peak": value / 2250.0,
         "ms_fwd_kernel": ms_f,
@@ -412,6 +426,8 @@ def run_ours(args):
     }
     if rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(w)
+        # the same kernels on the full causal set of the same shape
+        line["dense_causal"] = dense_comparator(st, w, ms_step)
     if rank == 0 and not args.no_extra and world == 1:
         line["workloads"] = extra_workloads(st, w.name)
     if world > 1:
@@ -463,15 +479,27 @@ def time_workload(st, w, steps=5, warmup=2, kind=None):
     assert st.st_last_device_status() == st.ST_OK
     nnz = nnz_of(L, w)
     ms = statistics.mean(tot)
-    peaks, _ = load_peaks()
+    peaks, peak_src = load_peaks()
     flops = 14.0 * w.d * nnz
     return {"ms_step": ms, "ms_fwd_kernel": statistics.mean(tf),
             "ms_bwd_kernel": statistics.mean(tb), "nnz": nnz,
             "useful_tflops": flops / (ms * 1e-3) / 1e12,
             "pct_of_peak": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
             "step_roofline": step_roofline(w, flops, ms, peaks),
+            "roofline": kernel_roofline(w, nnz, statistics.mean(tb), peaks, peak_src),
             "fwd_tflops": 4.0 * w.d * nnz / (statistics.mean(tf) * 1e-3) / 1e12,
             "bwd_kernel_tflops": 10.0 * w.d * nnz / (statistics.mean(tb) * 1e-3) / 1e12}
+
+
+def dense_comparator(st, w, sparse_ms):
+    """The same kernels on the full causal set of the workload's shape: its
+    time per fwd + bwd step, useful TFLOP/s over its own (causal) pairs, and
+    how much faster the sparse step is."""
+    steps, warmup = (3, 1) if w.T >= 32768 else (5, 2)
+    r = time_workload(st, w, steps=steps, warmup=warmup, kind="dense")
+    return {"ms_step": r["ms_step"], "useful_tflops": r["useful_tflops"],
+            "ms_fwd_kernel": r["ms_fwd_kernel"], "ms_bwd_kernel": r["ms_bwd_kernel"],
+            "nnz": r["nnz"], "sparse_speedup": r["ms_step"] / sparse_ms}
 
 
 def extra_workloads(st, skip):
@@ -480,9 +508,10 @@ def extra_workloads(st, skip):
         w = synth.WORKLOADS[name]
         if name == skip or w.dtype != "bf16":
             continue
-        out[name] = time_workload(st, w)
-    w = synth.WORKLOADS["strided-merged-T65536"]
-    out["dense-causal-T65536"] = time_workload(st, w, steps=3, warmup=1, kind="dense")
+        r = time_workload(st, w)
+        r["dense_causal"] = dense_comparator(st, w, r["ms_step"])
+        r["cpu_baseline"] = cpu_baseline(w, budget_s=6.0)
+        out[name] = r
     return out
 
 
@@ -515,8 +544,8 @@ def oracle_sample(w, budget_s=15.0):
     return run, nh, nnz, threads, t2
 
 
-def cpu_baseline(w):
-    run, nh, nnz, threads, _ = oracle_sample(w)
+def cpu_baseline(w, budget_s=15.0):
+    run, nh, nnz, threads, _ = oracle_sample(w, budget_s=budget_s)
     t = run(nh)
     return {"value": 14.0 * w.d * nnz / t / 1e12, "unit": "TFLOP/s", "cores": threads,
             "kind": "oracle",
@@ -540,7 +569,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name, "sampled_heads": nh},
+            "data": "synthetic", "config": workload_config(w, args.gpus),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
