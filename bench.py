@@ -316,6 +316,7 @@ def run_ours(args):
     # per-kernel times for the roofline: eager steps with the library's own
     # events around the attention kernels, on the stream they run on
     st.st_kernel_timing(True)
+    kp, kn = [], []
     for _ in range(args.steps):
         flush.zero_()
         torch.cuda._sleep(400000)  # the host queues the whole step before the GPU reaches it
@@ -323,6 +324,9 @@ def run_ours(args):
         torch.cuda.synchronize()
         kf.append(st.st_kernel_elapsed_ms(0))
         kb.append(st.st_kernel_elapsed_ms(1))
+        if dt_code != st.ST_F32:
+            kp.append(st.st_kernel_elapsed_ms(2))
+            kn.append(st.st_kernel_elapsed_ms(3))
     st.st_kernel_timing(False)
     del graph
     total_ms = max_over_ranks(sum(times), dev)
@@ -410,6 +414,8 @@ def run_ours(args):
         "pct_of_spec_peak": value / 2250.0,
         "ms_fwd_kernel": ms_f,
         "ms_bwd_kernel": ms_b,
+        "ms_bwd_prologue": statistics.mean(kp) if kp else None,
+        "ms_bwd_epilogue": statistics.mean(kn) if kn else None,
         "nnz": nnz,
         "useful_flops_per_step": flops,
         # the same step counted without the backward's recomputation of S
@@ -468,6 +474,7 @@ def time_workload(st, w, steps=5, warmup=2, kind=None):
         tot.append(e0.elapsed_time(e1))
     del graph
     st.st_kernel_timing(True)
+    tp, tn = [], []
     for _ in range(steps):
         flush.zero_()
         torch.cuda._sleep(400000)  # the host queues the whole step before the GPU reaches it
@@ -475,6 +482,8 @@ def time_workload(st, w, steps=5, warmup=2, kind=None):
         torch.cuda.synchronize()
         tf.append(st.st_kernel_elapsed_ms(0))
         tb.append(st.st_kernel_elapsed_ms(1))
+        tp.append(st.st_kernel_elapsed_ms(2))
+        tn.append(st.st_kernel_elapsed_ms(3))
     st.st_kernel_timing(False)
     assert st.st_last_device_status() == st.ST_OK
     nnz = nnz_of(L, w)
@@ -482,7 +491,8 @@ def time_workload(st, w, steps=5, warmup=2, kind=None):
     peaks, peak_src = load_peaks()
     flops = 14.0 * w.d * nnz
     return {"ms_step": ms, "ms_fwd_kernel": statistics.mean(tf),
-            "ms_bwd_kernel": statistics.mean(tb), "nnz": nnz,
+            "ms_bwd_kernel": statistics.mean(tb), "ms_bwd_prologue": statistics.mean(tp),
+            "ms_bwd_epilogue": statistics.mean(tn), "nnz": nnz,
             "useful_tflops": flops / (ms * 1e-3) / 1e12,
             "pct_of_peak": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
             "step_roofline": step_roofline(w, flops, ms, peaks),

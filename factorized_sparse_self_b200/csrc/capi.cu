@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -17,8 +18,9 @@ using namespace st;
 namespace {
 
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;
-uint64_t g_wait_ns = kDefaultWaitNs;
-int g_force_timeout = 0;
+// Process-wide, read by every later launch from any host thread.
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+std::atomic<int> g_force_timeout{0};
 
 constexpr int kMaxDevices = 64;
 int* g_status[kMaxDevices] = {nullptr};
@@ -63,8 +65,10 @@ void free_device(st_layout* L) {
   for (int f = 1; f < 3; ++f) cudaFree(L->dev.bwd_split[f]);
   cudaFree(L->dev.sched_slots);
   cudaFree(L->dev.q_ents);
-  for (int hc = 0; hc < 2; ++hc)
+  for (int hc = 0; hc < 2; ++hc) {
     for (int k = 0; k < N_ROWLISTS; ++k) cudaFree(L->dev.rows[hc][k]);
+    for (int k = 0; k < 2; ++k) cudaFree(L->dev.segs[hc][k]);
+  }
   if (prev >= 0) cudaSetDevice(prev);
   L->on_device = false;
 }
@@ -103,7 +107,7 @@ st_status prepare(const st_layout* L, st_dtype dtype, int32_t B, int32_t H, int3
   c.scale = (scale > 0.f) ? scale : 1.0f / sqrtf((float)d);
   c.nclasses = nclasses;
   c.status = status_word(dev, false);
-  c.wait_ns = g_wait_ns;
+  c.wait_ns = g_wait_ns.load();
   c.stream = reinterpret_cast<cudaStream_t>(stream);
   if (!c.status) return ST_ERR_CUDA;
   return ST_OK;
@@ -112,9 +116,12 @@ st_status prepare(const st_layout* L, st_dtype dtype, int32_t B, int32_t H, int3
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Benchmark instrumentation (st_kernel_timing).
+// Kernels with a pair of events: 0 forward attention launches, 1 backward
+// main kernel, 2 backward prologue, 3 backward epilogue.
+constexpr int kTimed = 4;
 bool g_timing = false;
-cudaEvent_t g_ev[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
-bool g_ev_used[2] = {false, false};
+cudaEvent_t g_ev[kTimed][2] = {};
+bool g_ev_used[kTimed] = {};
 
 // Hands the benchmark events of `kernel` to a call (when timing is on).
 void arm(Call& c, int kernel) {
@@ -197,6 +204,11 @@ st_status st_pattern_layout(const st_pattern_desc* desc, st_layout** out, void* 
     for (int k = 0; k < N_ROWLISTS && e == cudaSuccess; ++k) {
       e = upload(&L->dev.rows[hc][k], L->rows[hc][k], cs);
       L->dev.n_rows[hc][k] = (int32_t)L->rows[hc][k].size();
+    }
+  for (int hc = 0; hc < (int)L->hcs.size() && e == cudaSuccess; ++hc)
+    for (int k = 0; k < 2 && e == cudaSuccess; ++k) {
+      e = upload(&L->dev.segs[hc][k], L->segs[hc][k], cs);
+      L->dev.n_segs[hc][k] = (int32_t)L->segs[hc][k].size();
     }
   if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
   if (e != cudaSuccess) {
@@ -302,9 +314,7 @@ st_status st_sparse_attn_fwd_heads(const st_layout* L, st_dtype dtype, int32_t B
   if (dtype == ST_F32) {
     e = simt_fwd(c, q, k, v, o, lse);
   } else {
-    int ft = g_force_timeout;
-    g_force_timeout = 0;
-    e = tc_fwd(c, q, k, v, o, lse, ft);
+    e = tc_fwd(c, q, k, v, o, lse, g_force_timeout.exchange(0));
   }
   return e == cudaSuccess ? ST_OK : ST_ERR_CUDA;
 }
@@ -371,13 +381,19 @@ st_status st_sparse_attn_bwd_heads(const st_layout* L, st_dtype dtype, int32_t B
     int* counter = reinterpret_cast<int*>(dv_acc + stride);  // work counter of the kernel
     float* slots = reinterpret_cast<float*>(reinterpret_cast<char*>(counter) + 256);
     int nslots = 0;
-    e = bwd_prep(c, o, dout, Dv, dq_acc, dk_acc, dv_acc, counter, slots, &nslots);
-    Call cm = c;
+    Call cp = c, cm = c, cf = c;
+    arm(cp, 2);
     arm(cm, 1);
+    arm(cf, 3);
+    record_begin(cp);
+    e = bwd_prep(c, o, dout, Dv, dq_acc, dk_acc, dv_acc, counter, slots, &nslots);
+    record_end(cp);
     if (e == cudaSuccess)
       e = tc_bwd(cm, q, k, v, lse, dout, Dv, dq_acc, dk_acc, dv_acc, dq, dk, dv, counter, slots,
                  nslots);
+    record_begin(cf);
     if (e == cudaSuccess) e = bwd_finish(c, dq_acc, dk_acc, dv_acc, slots, nslots, dq, dk, dv);
+    record_end(cf);
   }
   return e == cudaSuccess ? ST_OK : ST_ERR_CUDA;
 }
@@ -412,17 +428,17 @@ st_status st_layout_launches(const st_layout* L, st_dtype dtype, int32_t* fwd, i
 
 st_status st_kernel_timing(int32_t enable) {
   if (enable) {
-    for (int k = 0; k < 2; ++k)
+    for (int k = 0; k < kTimed; ++k)
       for (int w = 0; w < 2; ++w)
         if (!g_ev[k][w] && cudaEventCreate(&g_ev[k][w]) != cudaSuccess) return ST_ERR_CUDA;
-    g_ev_used[0] = g_ev_used[1] = false;
+    for (int k = 0; k < kTimed; ++k) g_ev_used[k] = false;
   }
   g_timing = enable != 0;
   return ST_OK;
 }
 
 st_status st_kernel_elapsed_ms(int32_t kernel, float* ms) {
-  if (kernel < 0 || kernel > 1 || !ms || !g_ev[kernel][1] || !g_ev_used[kernel])
+  if (kernel < 0 || kernel >= kTimed || !ms || !g_ev[kernel][1] || !g_ev_used[kernel])
     return ST_ERR_INVALID;
   if (cudaEventSynchronize(g_ev[kernel][1]) != cudaSuccess) return ST_ERR_CUDA;
   if (cudaEventElapsedTime(ms, g_ev[kernel][0], g_ev[kernel][1]) != cudaSuccess)
@@ -431,8 +447,8 @@ st_status st_kernel_elapsed_ms(int32_t kernel, float* ms) {
 }
 
 st_status st_set_wait_limit(uint64_t ns, int32_t force_timeout) {
-  g_wait_ns = ns ? ns : kDefaultWaitNs;
-  g_force_timeout = force_timeout ? 1 : 0;
+  g_wait_ns.store(ns ? ns : kDefaultWaitNs);
+  g_force_timeout.store(force_timeout ? 1 : 0);
   return ST_OK;
 }
 

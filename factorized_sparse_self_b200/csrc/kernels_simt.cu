@@ -273,29 +273,41 @@ __global__ void prologue_kernel(const E* __restrict__ o, const E* __restrict__ d
     acc[t] = z;
 }
 
-struct RowSet {
-  const int32_t* rows[2][N_ROWLISTS];
-  int32_t n[2][N_ROWLISTS];
+// Segments of the accumulated rows, per head class: [hc][0] dQ rows,
+// [hc][1] dK / dV rows (see RowSeg).
+struct SegSet {
+  const RowSeg* segs[2][2];
+  int32_t n[2][2];
 };
 
-// Row list k of head class hc, picked without dynamic indexing of the
+// Segment list k of head class hc, picked without dynamic indexing of the
 // parameter (which would copy it to local memory).
-__device__ __forceinline__ const int32_t* rows_of(const RowSet& rs, int hc, int k, int& n) {
-  n = hc ? rs.n[1][k] : rs.n[0][k];
-  return hc ? rs.rows[1][k] : rs.rows[0][k];
+__device__ __forceinline__ const RowSeg* segs_of(const SegSet& ss, int hc, int k, int& n) {
+  if (hc) {
+    n = k ? ss.n[1][1] : ss.n[1][0];
+    return k ? ss.segs[1][1] : ss.segs[1][0];
+  }
+  n = k ? ss.n[0][1] : ss.n[0][0];
+  return k ? ss.segs[0][1] : ss.segs[0][0];
 }
 
-RowSet row_set_of(const st_layout* L) {
-  RowSet r;
+SegSet seg_set_of(const st_layout* L) {
+  SegSet r;
   for (int hc = 0; hc < 2; ++hc)
-    for (int k = 0; k < N_ROWLISTS; ++k) {
-      r.rows[hc][k] = (const int32_t*)L->dev.rows[hc][k];
-      r.n[hc][k] = L->dev.n_rows[hc][k];
+    for (int k = 0; k < 2; ++k) {
+      r.segs[hc][k] = (const RowSeg*)L->dev.segs[hc][k];
+      r.n[hc][k] = L->dev.n_segs[hc][k];
     }
   return r;
 }
 
-// Grid (x, B*H); d = 64 bf16 rows of 128 bytes.
+// Flat head index of the y-th selected head (heads h0 .. h0+hn-1 of every
+// batch entry).
+__device__ __forceinline__ int sel_head(int y, const Heads& hs) {
+  const int b = fdiv(y, hs.fhn);
+  return b * hs.H + hs.h0 + (y - b * hs.hn);
+}
+
 // Dot product of eight 16-bit values (fp16 if F16, else bf16), in fp32.
 template <bool F16>
 __device__ __forceinline__ float dot8(const uint4& a, const uint4& b) {
@@ -326,72 +338,72 @@ __device__ __forceinline__ uint32_t absmax8_bf16(const uint4& a) {
   return max(x & 0xffffu, x >> 16);
 }
 
-// Backward prologue of the 16-bit path. Grid (bx, gy): blockIdx.x strides over
-// the rows of one head, blockIdx.y over the selected heads of every batch
-// entry (gy <= kDoutSlots / bx). Writes D_i = dout_i . O_i for every row,
-// zeroes the fp32 accumulator rows that collect several contributions and
-// the backward kernel's work counter, and (bf16) the largest |dout| seen by
-// each block into slots[blockIdx.y * gridDim.x + blockIdx.x], from which the
-// backward kernel takes the power-of-two scale of its fp16 copy of dout.
+// Backward prologue of the 16-bit path (rows of d = 64 16-bit values, 128
+// bytes). Its work comes in items of one warp, dealt round robin: for every
+// selected head, D_i = dout_i . O_i of its rows in blocks of 32, then its
+// accumulated dQ row segments and dK / dV row segments, zeroed. Each item is
+// one contiguous run of memory with all of a lane's loads in flight at once
+// (16 of 16 bytes for D), so the kernel streams. Also zeroes the backward
+// kernel's work counter and (bf16) writes the largest |dout| the block read
+// into slots[blockIdx.x], from which the backward kernel takes the
+// power-of-two scale of its fp16 copy of dout.
 template <bool F16>
-__global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
-                                float* __restrict__ Dv,
-                                int T, Heads hs, RowSet rs, float4* __restrict__ dq_acc,
-                                float4* __restrict__ dk_acc, float4* __restrict__ dv_acc,
-                                int* __restrict__ sched_counter, float* __restrict__ slots) {
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *sched_counter = 0;
-  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
-  const int stride = gridDim.x * blockDim.x;
+__global__ void __launch_bounds__(256, 3)
+bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
+                float* __restrict__ Dv, int T, Heads hs, SegSet ss, int maxq, int maxk,
+                float4* __restrict__ dq_acc, float4* __restrict__ dk_acc,
+                float4* __restrict__ dv_acc, int* __restrict__ sched_counter,
+                float* __restrict__ slots) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *sched_counter = 0;
   const int lane = threadIdx.x & 31, sub = lane & 7;
-  const int nheads = hs.B * hs.hn;
+  const int rblocks = T / 32;  // T is a multiple of 128
+  const int per_head = rblocks + maxq + maxk;
+  const long long items = (long long)hs.B * hs.hn * per_head;
+  const int nw = (int)((gridDim.x * blockDim.x) >> 5);
+  const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
   uint32_t amax = 0;  // bf16 bits of the largest |dout| this thread read
-  for (int y = blockIdx.y; y < nheads; y += gridDim.y) {
-    const int bh = (y / hs.hn) * hs.H + hs.h0 + y % hs.hn;
-    const int hc = class_of(bh, hs);
+  for (long long w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < items; w += nw) {
+    const int y = (int)(w / per_head);
+    const int k = (int)(w - (long long)y * per_head);
+    const int bh = sel_head(y, hs);
     const size_t rb = (size_t)bh * T;
-    // D: eight lanes per 128-byte row (one 16-byte chunk each), four rows per
-    // warp and pass, four passes' loads in flight per thread
-    {
-      const int rstep = stride >> 3;  // rows per pass over the grid (multiple of 4)
-      const uint4* o4 = o + rb * 8;
-      const uint4* d4 = dout + rb * 8;
-      for (int rw = (tid >> 5) * 4; rw < T; rw += 4 * rstep) {  // warp-uniform
-        uint4 a[4], b[4];
+    if (k < rblocks) {
+      // rows 32k .. 32k+31: eight lanes per row (one 16-byte chunk each),
+      // rows (lane >> 3) + 4u for u = 0 .. 7
+      const size_t r0 = rb + 32 * (size_t)k;
+      uint4 a[8], b[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int r = rw + (lane >> 3) + u * rstep;
-          a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
-          if (r < T) {
-            a[u] = __ldg(o4 + (size_t)r * 8 + sub);
-            b[u] = __ldg(d4 + (size_t)r * 8 + sub);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if constexpr (!F16) amax = max(amax, absmax8_bf16(b[u]));
-          float sacc = dot8<F16>(a[u], b[u]);
-          sacc += __shfl_xor_sync(0xffffffffu, sacc, 4);
-          sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
-          sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
-          const int r = rw + (lane >> 3) + u * rstep;
-          if (sub == 0 && r < T) Dv[rb + r] = sacc;
-        }
+      for (int u = 0; u < 8; ++u) {
+        const size_t at = (r0 + (lane >> 3) + 4 * u) * 8 + sub;
+        a[u] = __ldg(o + at);
+        b[u] = __ldg(dout + at);
       }
-    }
-    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    {
-      int nr;
-      const int32_t* rows = rows_of(rs, hc, ROWS_Q_ACC, nr);
-      for (int64_t x = tid; x < (int64_t)nr * 16; x += stride)
-        dq_acc[(rb + rows[x >> 4]) * 16 + (x & 15)] = z4;
-    }
-    {
-      int nr;
-      const int32_t* rows = rows_of(rs, hc, ROWS_K_ACC, nr);
-      for (int64_t x = tid; x < (int64_t)nr * 16; x += stride) {
-        const size_t e = (rb + rows[x >> 4]) * 16 + (x & 15);
-        dk_acc[e] = z4;
-        dv_acc[e] = z4;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if constexpr (!F16) amax = max(amax, absmax8_bf16(b[u]));
+        float sacc = dot8<F16>(a[u], b[u]);
+        sacc += __shfl_xor_sync(0xffffffffu, sacc, 4);
+        sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
+        sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
+        if (sub == 0) Dv[r0 + (lane >> 3) + 4 * u] = sacc;
+      }
+    } else {
+      const int kk = k - rblocks;
+      const int isk = kk >= maxq ? 1 : 0;
+      int n;
+      const RowSeg* sg = segs_of(ss, class_of(bh, hs), isk, n);
+      const int si = isk ? kk - maxq : kk;
+      if (si >= n) continue;
+      const RowSeg seg = sg[si];
+      const size_t e0 = (rb + seg.start) * 16;  // float4 index of the segment's first row
+      const int ne = seg.len * 16;
+      if (isk) {
+        for (int x = lane; x < ne; x += 32) {
+          dk_acc[e0 + x] = z4;
+          dv_acc[e0 + x] = z4;
+        }
+      } else {
+        for (int x = lane; x < ne; x += 32) dq_acc[e0 + x] = z4;
       }
     }
   }
@@ -403,7 +415,7 @@ __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __rest
   if (threadIdx.x == 0) {
     uint32_t m = 0;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = max(m, wmax[w]);
-    slots[blockIdx.y * gridDim.x + blockIdx.x] = __uint_as_float(m << 16);
+    slots[blockIdx.x] = __uint_as_float(m << 16);
   }
 }
 
@@ -424,45 +436,65 @@ __device__ __forceinline__ uint4 round8f(const float4& a, const float4& b, float
                     round2<F16>(b.x * s, b.y * s), round2<F16>(b.z * s, b.w * s));
 }
 
-// Rounds the accumulated rows: eight elements (two float4 in, 16 bytes out)
-// per thread and step. dV partials carry the factor 2^e of the backward's
+// Rounds the accumulated rows into the 16-bit outputs: items of one warp,
+// one row segment of one selected head each (dQ segments first, then dK / dV
+// segments), with a lane's 16 loads of 16 bytes in flight at once. dQ and dK
+// take the softmax scale; dV partials carry the factor 2^e of the backward's
 // fp16 dout (from the prologue's slots; nslots = 0 means e = 0).
+// One row segment of an accumulator rounded into a 16-bit output, by one
+// warp: float4 pair p (eight elements, one 16-byte output) for p = lane +
+// 32 i, all loads in flight before the first store.
 template <bool F16>
-__global__ void bwd_finish_kernel(const float4* __restrict__ dq_acc,
-                                  const float4* __restrict__ dk_acc,
-                                  const float4* __restrict__ dv_acc, int T, Heads hs,
-                                  RowSet rs, float scale, const float* __restrict__ slots,
-                                  int nslots, uint4* __restrict__ dq,
-                                  uint4* __restrict__ dk, uint4* __restrict__ dv) {
+__device__ __forceinline__ void round_seg(const float4* __restrict__ acc, uint4* __restrict__ out,
+                                          size_t p0, int np, float sc, int lane) {
+  float4 a[8], b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int p = min(lane + 32 * i, np - 1);  // lanes past the end reload the last pair
+    a[i] = __ldg(acc + 2 * (p0 + p));
+    b[i] = __ldg(acc + 2 * (p0 + p) + 1);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (lane + 32 * i < np) out[p0 + lane + 32 * i] = round8f<F16>(a[i], b[i], sc);
+}
+
+template <bool F16>
+__global__ void __launch_bounds__(256, 2)
+bwd_finish_kernel(const float4* __restrict__ dq_acc, const float4* __restrict__ dk_acc,
+                  const float4* __restrict__ dv_acc, int T, Heads hs, SegSet ss, int maxq,
+                  int maxk, float scale, const float* __restrict__ slots, int nslots,
+                  uint4* __restrict__ dq, uint4* __restrict__ dk, uint4* __restrict__ dv) {
   __shared__ float bmax[32];
   float m = 0.f;
-  for (int s = threadIdx.x; s < nslots; s += blockDim.x) m = fmaxf(m, __ldg(slots + s));
+  for (int x = threadIdx.x; x < nslots; x += blockDim.x) m = fmaxf(m, __ldg(slots + x));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
   if ((threadIdx.x & 31) == 0) bmax[threadIdx.x >> 5] = m;
   __syncthreads();
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, bmax[w]);
   const float dv_scale = pow2f(-dout_exp(m));
-  const int bh = (blockIdx.y / hs.hn) * hs.H + hs.h0 + blockIdx.y % hs.hn;
-  const int hc = class_of(bh, hs);
-  const size_t rb = (size_t)bh * T;
-  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
-  const int stride = gridDim.x * blockDim.x;
-  {
-    int nr;
-    const int32_t* rows = rows_of(rs, hc, ROWS_Q_ACC, nr);
-    for (int64_t x = tid; x < (int64_t)nr * 8; x += stride) {
-      const size_t e = (rb + rows[x >> 3]) * 8 + (x & 7);
-      dq[e] = round8f<F16>(__ldg(dq_acc + 2 * e), __ldg(dq_acc + 2 * e + 1), scale);
-    }
-  }
-  {
-    int nr;
-    const int32_t* rows = rows_of(rs, hc, ROWS_K_ACC, nr);
-    for (int64_t x = tid; x < (int64_t)nr * 8; x += stride) {
-      const size_t e = (rb + rows[x >> 3]) * 8 + (x & 7);
-      dk[e] = round8f<F16>(__ldg(dk_acc + 2 * e), __ldg(dk_acc + 2 * e + 1), scale);
-      dv[e] = round8f<F16>(__ldg(dv_acc + 2 * e), __ldg(dv_acc + 2 * e + 1), dv_scale);
+  const int lane = threadIdx.x & 31;
+  const int per_head = maxq + maxk;
+  const long long items = (long long)hs.B * hs.hn * per_head;
+  const int nw = (int)((gridDim.x * blockDim.x) >> 5);
+  for (long long w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < items; w += nw) {
+    const int y = (int)(w / per_head);
+    const int k = (int)(w - (long long)y * per_head);
+    const int bh = sel_head(y, hs);
+    const int isk = k >= maxq ? 1 : 0;
+    int n;
+    const RowSeg* sg = segs_of(ss, class_of(bh, hs), isk, n);
+    const int si = isk ? k - maxq : k;
+    if (si >= n) continue;
+    const RowSeg seg = sg[si];
+    const size_t p0 = ((size_t)bh * T + seg.start) * 8;
+    const int np = seg.len * 8;  // at most 256: eight per lane
+    if (isk) {
+      round_seg<F16>(dk_acc, dk, p0, np, scale, lane);
+      round_seg<F16>(dv_acc, dv, p0, np, dv_scale, lane);
+    } else {
+      round_seg<F16>(dq_acc, dq, p0, np, scale, lane);
     }
   }
 }
@@ -571,23 +603,33 @@ cudaError_t bwd_prologue(const Call& c, const void* o, const void* dout, float* 
   return cudaGetLastError();
 }
 
-int prep_grid(const Call& c, dim3& grid) {
-  const int T = c.L->geom.T;
-  const int bx = std::max(1, std::min(64, (T + 127) / 128));
-  const int gy = std::max(1, std::min(c.B * c.hn, kDoutSlots / bx));
-  grid = dim3(bx, gy);
-  return bx * gy;
+// Largest segment counts over the head classes: dQ rows, dK / dV rows.
+void max_segs(const st_layout* L, int& maxq, int& maxk) {
+  maxq = maxk = 0;
+  for (int hc = 0; hc < (int)L->hcs.size(); ++hc) {
+    maxq = std::max(maxq, L->dev.n_segs[hc][0]);
+    maxk = std::max(maxk, L->dev.n_segs[hc][1]);
+  }
+}
+
+// Blocks of 8 warps for `items` warp items, at most `cap`.
+int warp_grid(long long items, int cap) {
+  return (int)std::max<long long>(1, std::min<long long>((items + 7) / 8, cap));
 }
 
 cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* Dv, float* dq_acc,
                      float* dk_acc, float* dv_acc, int* sched_counter, float* slots,
                      int* nslots) {
-  dim3 grid;
-  *nslots = prep_grid(c, grid);
+  const int T = c.L->geom.T;
+  int maxq, maxk;
+  max_segs(c.L, maxq, maxk);
+  const long long items = (long long)c.B * c.hn * (T / 32 + maxq + maxk);
+  const int grid = warp_grid(items, std::min(kDoutSlots, sm_count() * 3));
+  *nslots = grid;
   auto kern = (c.dtype == ST_F16) ? bwd_prep_kernel<true> : bwd_prep_kernel<false>;
-  kern<<<grid, 256, 0, c.stream>>>(
-      (const uint4*)o, (const uint4*)dout, Dv, c.L->geom.T, heads_of(c),
-      row_set_of(c.L), (float4*)dq_acc, (float4*)dk_acc, (float4*)dv_acc, sched_counter, slots);
+  kern<<<grid, 256, 0, c.stream>>>((const uint4*)o, (const uint4*)dout, Dv, T, heads_of(c),
+                                   seg_set_of(c.L), maxq, maxk, (float4*)dq_acc,
+                                   (float4*)dk_acc, (float4*)dv_acc, sched_counter, slots);
   return cudaGetLastError();
 }
 
@@ -595,17 +637,16 @@ cudaError_t bwd_finish(const Call& c, const float* dq_acc, const float* dk_acc,
                        const float* dv_acc, const float* slots, int nslots, void* dq, void* dk,
                        void* dv) {
   const st_layout* L = c.L;
-  int most = 0;
-  for (int hc = 0; hc < (int)L->hcs.size(); ++hc)
-    most = std::max(most, std::max(L->dev.n_rows[hc][ROWS_Q_ACC], L->dev.n_rows[hc][ROWS_K_ACC]));
-  if (most == 0) return cudaSuccess;  // every row was written directly
-  const int bx = std::max(1, std::min(64, (most + 31) / 32));
-  dim3 grid(bx, c.B * c.hn);
+  int maxq, maxk;
+  max_segs(L, maxq, maxk);
+  if (maxq + maxk == 0) return cudaSuccess;  // every row was written directly
+  const long long items = (long long)c.B * c.hn * (maxq + maxk);
+  const int grid = warp_grid(items, sm_count() * 2);
   auto kern = (c.dtype == ST_F16) ? bwd_finish_kernel<true> : bwd_finish_kernel<false>;
   kern<<<grid, 256, 0, c.stream>>>(
       (const float4*)dq_acc, (const float4*)dk_acc, (const float4*)dv_acc, L->geom.T,
-      heads_of(c), row_set_of(L), c.scale, slots, c.dtype == ST_F16 ? 0 : nslots, (uint4*)dq,
-      (uint4*)dk, (uint4*)dv);
+      heads_of(c), seg_set_of(L), maxq, maxk, c.scale, slots, c.dtype == ST_F16 ? 0 : nslots,
+      (uint4*)dq, (uint4*)dk, (uint4*)dv);
   return cudaGetLastError();
 }
 

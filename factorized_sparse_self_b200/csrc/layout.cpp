@@ -258,6 +258,18 @@ void assign_writers(st_layout* L) {
       if (wq[(size_t)t] == 0) L->rows[hc][ROWS_Q_ZERO].push_back(t);
       if (wk[(size_t)t] == 0) L->rows[hc][ROWS_K_ZERO].push_back(t);
     }
+    // the accumulated rows as runs of consecutive rows, cut at kSegRows
+    for (int k = 0; k < 2; ++k) {
+      const std::vector<int32_t>& rl = L->rows[hc][k ? ROWS_K_ACC : ROWS_Q_ACC];
+      std::vector<RowSeg>& sg = L->segs[hc][k];
+      sg.clear();
+      for (size_t a = 0; a < rl.size();) {
+        size_t b = a + 1;
+        while (b < rl.size() && rl[b] == rl[b - 1] + 1 && (int)(b - a) < kSegRows) ++b;
+        sg.push_back(RowSeg{rl[a], (int32_t)(b - a)});
+        a = b;
+      }
+    }
   }
 }
 

@@ -90,6 +90,14 @@ enum RowList : int {
   N_ROWLISTS = 4
 };
 
+// The accumulated rows (ROWS_Q_ACC, ROWS_K_ACC) as segments of consecutive
+// rows, at most kSegRows each: the backward prologue zeroes and the epilogue
+// rounds one segment per warp, as a contiguous run of memory.
+constexpr int kSegRows = 32;
+struct RowSeg {
+  int32_t start, len;
+};
+
 // Heads a call covers: heads h0 .. h0+hn-1 of tensors with B x H heads, for a
 // layout with nclasses head classes (kernel parameter, plain old data).
 // Division by a divisor that is fixed for a launch, by a multiply-high and a
@@ -167,6 +175,9 @@ struct DeviceSchedule {
   void* rows[2][N_ROWLISTS] = {{nullptr, nullptr, nullptr, nullptr},
                                {nullptr, nullptr, nullptr, nullptr}};
   int32_t n_rows[2][N_ROWLISTS] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+  // per head class: segments of ROWS_Q_ACC (index 0) and ROWS_K_ACC (1)
+  void* segs[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+  int32_t n_segs[2][2] = {{0, 0}, {0, 0}};
 };
 
 }  // namespace st
@@ -184,6 +195,7 @@ struct st_layout {
   std::vector<st::BwdItem> bwd_split[2];  // parts of 2 and of 4 (see DeviceSchedule)
   std::vector<st::QEnt> q_ents;
   std::vector<int32_t> rows[2][st::N_ROWLISTS];  // see st::RowList
+  std::vector<st::RowSeg> segs[2][2];            // see st::RowSeg
   bool on_device = false;
   int device = -1;
   mutable std::atomic<uint32_t> next_slot{0};  // round robin over dev.sched_slots

@@ -130,7 +130,10 @@ st_status st_layout_export(const st_layout* layout, int32_t head_class, int32_t 
 /* Live pairs of one head of the class (sum over i of |S_i|). */
 st_status st_layout_nnz(const st_layout* layout, int32_t head_class, int64_t* nnz);
 
-/* Forward: O and LSE for all B*H heads. Head h = index within H of the
+/* Forward: O and LSE for all B*H heads ("Sparse Transformer" milestone page,
+ * nlp-lineage, "The idea", "The notation": O_i = softmax(q_i K_{S_i}^T / sqrt(d))
+ * V_{S_i}, normalised over S_i only, llm-arch-kb section 2, "Sparse attention
+ * as an unnormalized form"). Head h = index within H of the
  * [B, H, T, d] tensors (split mode picks A1/A2 from its parity). Rows with an
  * empty set get O = 0 and LSE = -inf. For a strided merged layout the call
  * runs two passes (natural-order window keys, then residue-order strided
@@ -146,12 +149,19 @@ st_status st_sparse_attn_fwd(const st_layout* layout, st_dtype dtype, int32_t B,
 st_status st_sparse_attn_bwd_workspace(const st_layout* layout, st_dtype dtype, int32_t B,
                                        int32_t H, int32_t T, int32_t d, size_t* bytes);
 
-/* Backward: dQ, dK, dV (dtype of the inputs, fp32 accumulation) from Q, K,
+/* Backward ("Sparse Transformer" milestone page, nlp-lineage, "The idea",
+ * "Recomputation": the attention matrix is rebuilt from the saved LSE rather
+ * than stored): dQ, dK, dV (dtype of the inputs, fp32 accumulation) from Q, K,
  * V, the forward's O and LSE, and the upstream gradient dout. P is recomputed
  * as exp(s - LSE) on live tiles; D_i = dout_i . O_i. The workspace (device
  * memory, at least st_sparse_attn_bwd_workspace bytes, 256-byte aligned) is
- * overwritten; it holds D, the fp32 accumulators and a work counter. Returns
- * ST_ERR_WORKSPACE if it is missing or too small. */
+ * overwritten; it holds D, the fp32 accumulators, a work counter and the
+ * prologue's per-block maxima of |dout|. Returns ST_ERR_WORKSPACE if it is
+ * missing or too small. On the 16-bit path dV is formed from P and dout in
+ * fp16 (dout times a power of two chosen from its largest magnitude), and
+ * rows with several contributions are summed by fp32 reduce-adds whose order
+ * varies: results are not bitwise reproducible from run to run (within one
+ * rounding step of the output type). */
 st_status st_sparse_attn_bwd(const st_layout* layout, st_dtype dtype, int32_t B, int32_t H,
                              int32_t T, int32_t d, float scale, const void* q, const void* k,
                              const void* v, const void* o, const float* lse, const void* dout,
@@ -216,10 +226,12 @@ st_status st_sparse_attn_bwd_noalloc(const st_layout* layout, st_dtype dtype, in
 st_status st_last_device_status(void* stream);
 
 /* Upper bound, in nanoseconds, of every on-device wait of later launches
- * (default 2e9). 0 restores the default. A wait that runs out sets the status
- * word and makes the kernel return early. For tests of the timeout path only,
- * force_timeout != 0 makes the next forward launch skip the loads of its
- * first key tile so its waits run out on purpose (the GPU stays usable). */
+ * (default 2e9), process-wide: it applies to launches from every host thread
+ * (the setting is atomic). 0 restores the default. A wait that runs out sets
+ * the status word and makes the kernel return early. For tests of the timeout
+ * path only, force_timeout != 0 makes the next bf16 / fp16 forward launch, from
+ * whichever thread comes first, skip the loads of its first key tile so its
+ * waits run out on purpose (the GPU stays usable). */
 st_status st_set_wait_limit(uint64_t ns, int32_t force_timeout);
 
 /* Kernel launches one fwd / bwd call makes with this layout and dtype (the
@@ -228,16 +240,20 @@ st_status st_set_wait_limit(uint64_t ns, int32_t force_timeout);
 st_status st_layout_launches(const st_layout* layout, st_dtype dtype, int32_t* fwd_launches,
                              int32_t* bwd_launches);
 
-/* Benchmark instrumentation. enable != 0 creates (once) two pairs of CUDA
+/* Benchmark instrumentation. enable != 0 creates (once) four pairs of CUDA
  * events on the current device; from then on every fwd call records pair 0
- * around its attention launches and every bwd call records pair 1 around its
- * main attention kernel, on the call's stream. enable = 0 stops recording.
- * Events are created here, never inside fwd/bwd. */
+ * around its attention launches, and every bwd call records pair 1 around its
+ * main attention kernel, pair 2 around its prologue and pair 3 around its
+ * epilogue (16-bit path; the epilogue pair brackets nothing when no row
+ * accumulates), on the call's stream. enable = 0 stops recording. Events are
+ * created here, never inside fwd/bwd. Not thread-safe: one host thread may
+ * time calls at a time. */
 st_status st_kernel_timing(int32_t enable);
 
 /* Milliseconds between the pair of events of the latest call of `kernel`
- * (0 = forward attention launches, 1 = backward main kernel); synchronises on
- * that call's stop event. ST_ERR_INVALID if timing is off or nothing ran. */
+ * (0 = forward attention launches, 1 = backward main kernel, 2 = backward
+ * prologue, 3 = backward epilogue); synchronises on that call's stop event.
+ * ST_ERR_INVALID if timing is off or nothing ran. */
 st_status st_kernel_elapsed_ms(int32_t kernel, float* ms);
 
 /* Static description of a status code. */
