@@ -5,9 +5,10 @@
 
 Prints one JSON line with per-call CUDA-event times of the forward attention
 launches, of the backward attention kernel and of the whole forward + backward
-call pair (ms_step), and the useful TFLOP/s (4 d nnz forward, 10 d nnz
-backward). --flush writes 256 MB between iterations so that every call starts
-with a cold L2. Inputs are the seeded synthetic ones
+call pair (ms_step), of the backward's prologue and epilogue kernels (16-bit
+inputs), and the useful TFLOP/s (4 d nnz forward, 10 d nnz backward).
+--flush writes 256 MB between iterations so that every call starts with a
+cold L2. Inputs are the seeded synthetic ones
 (bf16, std 0.5; dO ~ N(0, 1)).
 """
 from __future__ import annotations
@@ -66,7 +67,7 @@ def main():
     torch.cuda.synchronize()
     flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda") if a.flush else None
     st.st_kernel_timing(True)
-    tf, tb, ts = [], [], []
+    tf, tb, ts, tp, te = [], [], [], [], []
     for _ in range(a.iters):
         if flush is not None:
             flush.zero_()
@@ -81,6 +82,9 @@ def main():
         tf.append(st.st_kernel_elapsed_ms(0))
         if not a.fwd_only:
             tb.append(st.st_kernel_elapsed_ms(1))
+            if code != st.ST_F32:
+                tp.append(st.st_kernel_elapsed_ms(2))
+                te.append(st.st_kernel_elapsed_ms(3))
     st.st_kernel_timing(False)
     status = st.st_last_device_status()
     if status != st.ST_OK:
@@ -91,6 +95,10 @@ def main():
     if tb:
         res["ms_bwd_kernel"] = statistics.mean(tb)
         res["bwd_kernel_tflops"] = 10.0 * a.d * nnz / (statistics.mean(tb) * 1e-3) / 1e12
+    if tp:
+        res["ms_bwd_prologue"] = statistics.mean(tp)
+        res["ms_bwd_epilogue"] = statistics.mean(te)
+    res["flush"] = bool(a.flush)
     print(json.dumps(res), flush=True)
 
 
