@@ -340,13 +340,17 @@ __device__ __forceinline__ uint32_t absmax8_bf16(const uint4& a) {
 
 // Backward prologue of the 16-bit path (rows of d = 64 16-bit values, 128
 // bytes). Its work comes in items of one warp, dealt round robin: for every
-// selected head, D_i = dout_i . O_i of its rows in blocks of 32, then its
+// selected head, D_i = dout_i . O_i of its rows in blocks of 16, then its
 // accumulated dQ row segments and dK / dV row segments, zeroed. Each item is
 // one contiguous run of memory with all of a lane's loads in flight at once
-// (16 of 16 bytes for D), so the kernel streams. Also zeroes the backward
+// (8 of 16 bytes for D), so the kernel streams. Also zeroes the backward
 // kernel's work counter and (bf16) writes the largest |dout| the block read
 // into slots[blockIdx.x], from which the backward kernel takes the
 // power-of-two scale of its fp16 copy of dout.
+// Rows of a D item per group of eight lanes (items of 16 rows: more, smaller
+// items balance the warps better than 32-row ones did at T = 12288).
+constexpr int kDU = 4;
+
 template <bool F16>
 __global__ void __launch_bounds__(256, 3)
 bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
@@ -356,7 +360,8 @@ bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
                 float* __restrict__ slots) {
   if (blockIdx.x == 0 && threadIdx.x == 0) *sched_counter = 0;
   const int lane = threadIdx.x & 31, sub = lane & 7;
-  const int rblocks = T / 32;  // T is a multiple of 128
+  constexpr int kDRows = 4 * kDU;  // rows of one D item
+  const int rblocks = T / kDRows;  // T is a multiple of 128
   const int per_head = rblocks + maxq + maxk;
   const long long items = (long long)hs.B * hs.hn * per_head;
   const int nw = (int)((gridDim.x * blockDim.x) >> 5);
@@ -368,18 +373,18 @@ bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
     const int bh = sel_head(y, hs);
     const size_t rb = (size_t)bh * T;
     if (k < rblocks) {
-      // rows 32k .. 32k+31: eight lanes per row (one 16-byte chunk each),
-      // rows (lane >> 3) + 4u for u = 0 .. 7
-      const size_t r0 = rb + 32 * (size_t)k;
-      uint4 a[8], b[8];
+      // rows kDRows k .. kDRows (k+1) - 1: eight lanes per row (one 16-byte
+      // chunk each), rows (lane >> 3) + 4u for u < kDU
+      const size_t r0 = rb + kDRows * (size_t)k;
+      uint4 a[kDU], b[kDU];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < kDU; ++u) {
         const size_t at = (r0 + (lane >> 3) + 4 * u) * 8 + sub;
         a[u] = __ldg(o + at);
         b[u] = __ldg(dout + at);
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < kDU; ++u) {
         if constexpr (!F16) amax = max(amax, absmax8_bf16(b[u]));
         float sacc = dot8<F16>(a[u], b[u]);
         sacc += __shfl_xor_sync(0xffffffffu, sacc, 4);
@@ -450,9 +455,12 @@ __device__ __forceinline__ void round_seg(const float4* __restrict__ acc, uint4*
   float4 a[8], b[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int p = min(lane + 32 * i, np - 1);  // lanes past the end reload the last pair
-    a[i] = __ldg(acc + 2 * (p0 + p));
-    b[i] = __ldg(acc + 2 * (p0 + p) + 1);
+    const int p = lane + 32 * i;
+    a[i] = b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p < np) {
+      a[i] = __ldg(acc + 2 * (p0 + p));
+      b[i] = __ldg(acc + 2 * (p0 + p) + 1);
+    }
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i)
@@ -623,7 +631,7 @@ cudaError_t bwd_prep(const Call& c, const void* o, const void* dout, float* Dv, 
   const int T = c.L->geom.T;
   int maxq, maxk;
   max_segs(c.L, maxq, maxk);
-  const long long items = (long long)c.B * c.hn * (T / 32 + maxq + maxk);
+  const long long items = (long long)c.B * c.hn * (T / (4 * kDU) + maxq + maxk);
   const int grid = warp_grid(items, std::min(kDoutSlots, sm_count() * 3));
   *nslots = grid;
   auto kern = (c.dtype == ST_F16) ? bwd_prep_kernel<true> : bwd_prep_kernel<false>;
