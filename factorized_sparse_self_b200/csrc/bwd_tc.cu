@@ -58,12 +58,17 @@ static_assert(256 * kRegsCompute + 128 * kRegsIssue == kThreads * 168, "register
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
 constexpr uint32_t kColPT = 448;  // P^T as packed bf16 pairs, 64 columns
+// packed fp32 summary rows of one column half (kv_direct == 2 units), staged
+// in the dS^T buffer at the end of a unit: dK halves, then dV halves
+constexpr int kSumBoxBytes = kMixedMaxRows * 128;
+static_assert(4 * kSumBoxBytes <= 2 * kTileBytes, "summary-row boxes exceed the dS^T buffer");
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdMaps {
   CUtensorMap q[3], k[3], v[3], dout[3];  // bf16, indexed by View
   CUtensorMap dq[3], dk[3], dv[3];        // fp32 accumulators, 32-float boxes
   CUtensorMap dqo[3], dko[3], dvo[3];     // bf16 outputs (direct tiles)
+  CUtensorMap dks, dvs;  // fp32 accumulators: the summary rows of a natural tile
 };
 
 // A published work unit: its index (n_units: no more work), head, item and
@@ -143,6 +148,14 @@ __device__ __forceinline__ void reduce_half(const CUtensorMap* maps, int view, c
     int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_reduce_add_4d(&maps[VIEW_CLS], s, h * 32, r, pb * kTile, bh);
   }
+}
+
+// Reduce-adds column half h of the summary rows of natural key tile `tile`,
+// staged packed (one 128-byte row per summary row, block after block) at src.
+__device__ __forceinline__ void reduce_summary_rows(const CUtensorMap* map, const Geom& g,
+                                                    int tile, int bh, const uint8_t* src,
+                                                    int h) {
+  tma_reduce_add_4d(map, src, h * 32, g.l - g.c, fdiv(tile * kTile, g.fl), bh);
 }
 
 // Stores a 128-row bf16 tile (coordinates are never negative).
@@ -598,13 +611,21 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           ok = false;
           break;
         }
-        if (x.it.kv_direct) {  // both 16-bit tiles in kvst; dst was not used
-          if (lane == 0) mbar_arrive(&S.dst_free);
+        if (x.it.kv_direct) {  // both 16-bit tiles in kvst
           if (lane < 2) {
             store_tile(lane ? maps.dvo : maps.dko, x.it.kview, g, x.it.ktile, x.bh,
                        S.kvst + lane * kTileBytes);
             bulk_commit();
+          } else if (x.it.kv_direct == 2 && lane < 6) {
+            // the packed fp32 summary rows in dst: dK halves, then dV halves
+            const int q = lane - 2;
+            reduce_summary_rows(q < 2 ? &maps.dks : &maps.dvs, g, x.it.ktile, x.bh,
+                                S.dst + q * kSumBoxBytes, q & 1);
+            bulk_commit();
+            bulk_wait_read_all();
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.dst_free);
         } else {  // lanes 0, 1: dV halves (in dst), read first; lanes 2, 3: dK halves
           if (lane < 4) {
             reduce_half(lane < 2 ? maps.dv : maps.dk, x.it.kview, g, x.it.ktile, x.bh,
@@ -860,6 +881,22 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           round8<F16>(r + ch * 8, sc, o4);
           st_shared_v4(dst + swz128(row, ch), o4[0], o4[1], o4[2], o4[3]);
         }
+        if (it.kv_direct == 2 && j >= 0) {
+          // a summary row also goes out unscaled in fp32, packed: row
+          // (offset in its block - (l - c)) + c (block - the tile's first block)
+          const int jb = fdiv(j, g.fl), o = j - jb * g.l;
+          if (o >= g.l - g.c) {
+            const int rr = (o - (g.l - g.c)) + g.c * (jb - fdiv(it.ktile * kTile, g.fl));
+            const uint32_t sb = ds_addr + wg * 2 * kSumBoxBytes;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch)
+                st_shared_v4(sb + h * kSumBoxBytes + swz128(rr, ch), r[h * 32 + ch * 4 + 0],
+                             r[h * 32 + ch * 4 + 1], r[h * 32 + ch * 4 + 2],
+                             r[h * 32 + ch * 4 + 3]);
+          }
+        }
       } else {
 #pragma unroll
         for (int h = 0; h < 2; ++h)
@@ -908,6 +945,14 @@ cudaError_t tc_bwd_t(const Call& c, const void* q, const void* k, const void* v,
       !make_view_maps(maps.dko, dk, el, L->geom, BH, c.d) ||
       !make_view_maps(maps.dvo, dv, el, L->geom, BH, c.d))
     return cudaErrorInvalidValue;
+  if (L->summary_rows) {
+    if (!make_summary_rows_map(&maps.dks, dk_acc, L->geom, BH, c.d) ||
+        !make_summary_rows_map(&maps.dvs, dv_acc, L->geom, BH, c.d))
+      return cudaErrorInvalidValue;
+  } else {
+    maps.dks = maps.dk[VIEW_NAT];  // never used
+    maps.dvs = maps.dv[VIEW_NAT];
+  }
   const size_t smem = sizeof(SmemBwd);
   static_assert(sizeof(SmemBwd) <= 227 * 1024, "shared memory plan exceeds a CTA's 227 KB");
   static bool attr_set[64] = {false};

@@ -116,6 +116,13 @@ enum Elem : int { ELEM_BF16 = 0, ELEM_F16 = 1, ELEM_F32 = 2 };
 bool make_view_maps(CUtensorMap out[3], const void* base, int elem, const Geom& g, int BH,
                     int d);
 
+// Encodes the summary rows of one natural 128-row tile of an fp32 [B*H, T, d]
+// tensor (the fixed pattern's last c rows of each l-block the tile covers,
+// l dividing 128 or 128 dividing l): a 4-D map over (d, l, T / l, B*H) with a
+// 32 x c x max(1, 128 / l) box, 128-byte swizzle. False when the layout has
+// no summary view or the driver rejects it.
+bool make_summary_rows_map(CUtensorMap* out, const void* base, const Geom& g, int BH, int d);
+
 // Element type of a call's 16-bit tensors.
 inline int elem16(const Call& c) { return c.dtype == ST_F16 ? ELEM_F16 : ELEM_BF16; }
 

@@ -213,13 +213,31 @@ void tile_rows(uint8_t v, const Geom& g, int32_t tile, std::vector<int32_t>& out
   }
 }
 
-// Who writes each gradient row (bf16 path). A backward unit writes dK, dV of
-// its whole key tile, a (unit, query tile) pair writes dQ of the query tile.
-// A tile whose rows all have exactly one writer is written directly in bf16
-// by that writer; rows with several writers go through fp32 accumulators;
-// rows nobody writes are zero-filled.
+// Summary keys of the fixed pattern: the last c positions of each l-block.
+bool is_summary_pos(const Geom& g, i64 j) { return j % g.l >= g.l - g.c; }
+
+// A natural key tile whose summary rows form one box of the backward
+// kernel's summary-rows tensor map: c rows in each of the tile's
+// max(1, 128 / l) l-blocks (l divides 128, or 128 divides l and the tile is
+// the last of its block), at most kMixedMaxRows rows.
+bool summary_box_fits(const BwdItem& it, const Geom& g) {
+  if (it.kview != VIEW_NAT || g.nsum == 0) return false;
+  const i64 l = g.l;
+  if (l <= kTile) return kTile % l == 0 && g.c * (kTile / l) <= kMixedMaxRows;
+  return l % kTile == 0 && ((i64)(it.ktile + 1) * kTile) % l == 0 && g.c <= kMixedMaxRows;
+}
+
+// Who writes each gradient row (16-bit path). A backward unit writes dK, dV
+// of its whole key tile, a (unit, query tile) pair writes dQ of the query
+// tile. A tile whose rows all have exactly one writer is written directly by
+// that writer; rows with several writers go through fp32 accumulators; rows
+// nobody writes are zero-filled. A natural key tile whose only shared rows are
+// summary keys (the fixed pattern's block tiles, whose summary keys later
+// query blocks also read) is stored directly and adds its summary rows to the
+// accumulators, so that only those rows take the fp32 round trip.
 void assign_writers(st_layout* L) {
   const Geom& g = L->geom;
+  L->summary_rows = false;
   std::vector<int32_t> rows;
   for (int hc = 0; hc < (int)L->hcs.size(); ++hc) {
     std::vector<int32_t> wk((size_t)g.T, 0), wq((size_t)g.T, 0);
@@ -238,9 +256,19 @@ void assign_writers(st_layout* L) {
       tile_rows(it.kview, g, it.ktile, rows);
       bool direct = true;
       for (int32_t j : rows) direct = direct && wk[(size_t)j] == 1;
-      it.kv_direct = direct ? 1 : 0;
-      if (!direct)
-        for (int32_t j : rows) acck[(size_t)j] = 1;
+      uint8_t how = direct ? 1 : 0;
+      if (!direct && summary_box_fits(it, g)) {
+        bool shared_are_summary = true;
+        for (int32_t j : rows)
+          shared_are_summary = shared_are_summary && (wk[(size_t)j] == 1 || is_summary_pos(g, j));
+        if (shared_are_summary) how = 2;
+      }
+      it.kv_direct = how;
+      if (how == 2) L->summary_rows = true;
+      // every summary row of a kv_direct == 2 tile is reduce-added (the box
+      // covers them all), so all of them are accumulated and rounded
+      for (int32_t j : rows)
+        if (how == 0 || (how == 2 && is_summary_pos(g, j))) acck[(size_t)j] = 1;
       for (int32_t e = it.qbeg; e < it.qend; ++e) {
         QEnt& qe = L->q_ents[(size_t)e];
         tile_rows(it.qview, g, qe.qtile, rows);

@@ -69,9 +69,19 @@ struct BwdItem {
   uint8_t kview;
   uint8_t qview;
   uint8_t rule;
-  uint8_t kv_direct;   // 1: this unit alone produces dK, dV of its key tile rows
+  // How dK, dV of the key tile leave the unit (16-bit path): 0, an fp32
+  // reduce-add of the whole tile; 1, a 16-bit store (this unit alone writes
+  // every row); 2, a 16-bit store of the whole tile plus an fp32 reduce-add of
+  // its summary rows only (a natural key tile of the fixed pattern whose
+  // summary keys other units also reach: the epilogue rounds those rows from
+  // the accumulator over the stored values).
+  uint8_t kv_direct;
   uint8_t pad[3];
 };
+
+// Most summary rows of one natural key tile that a kv_direct == 2 unit
+// stages: c rows in each of the tile's max(1, 128 / l) l-blocks.
+constexpr int kMixedMaxRows = 64;
 
 struct QEnt {
   int32_t qtile;
@@ -188,6 +198,7 @@ struct st_layout {
   std::vector<st::HeadClass> hcs;
   int32_t n_passes = 1;      // forward passes (2 for merged strided with class view)
   bool tc_ok = false;        // every segment's rows are intervals (tensor-core path usable)
+  bool summary_rows = false; // some backward unit has kv_direct == 2
   // host copies of the schedule
   std::vector<st::FwdItem> fwd_items[2];
   std::vector<st::KeyEnt> key_ents;

@@ -73,8 +73,28 @@ bool encode_views(CUtensorMap out[3], const void* base, int elem, const Geom& g,
   return true;
 }
 
+// The summary rows of one natural 128-row tile of an fp32 [B*H, T, d]
+// accumulator (fixed pattern, l dividing 128 or 128 dividing l): the box is 32
+// columns by c rows by max(1, 128 / l) l-blocks, i.e. the last c rows of each
+// block the tile covers, packed block after block.
+bool encode_summary_rows(CUtensorMap* out, const void* base, const Geom& g, int BH, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || g.nsum == 0) return false;
+  const cuuint64_t row = (cuuint64_t)d * 4;
+  const cuuint32_t one[4] = {1, 1, 1, 1};
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)g.l, (cuuint64_t)(g.T / g.l), (cuuint64_t)BH};
+  cuuint64_t str[3] = {row, (cuuint64_t)g.l * row, (cuuint64_t)g.T * row};
+  const int bpt = g.l < kTile ? kTile / g.l : 1;
+  cuuint32_t box[4] = {32, (cuuint32_t)g.c, (cuuint32_t)bpt, 1};
+  return enc(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, str, box,
+             one, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 struct Key {
   const void* base;
+  int what;  // 0: the three views, 1: the summary-rows map (in maps[0])
   int elem, T, l, c, P, nsum, BH, d;
   bool operator==(const Key& o) const { return std::memcmp(this, &o, sizeof(Key)) == 0; }
 };
@@ -91,13 +111,12 @@ Entry g_cache[kCacheSize];
 uint64_t g_clock = 0;
 std::mutex g_cache_mu;
 
-}  // namespace
-
-bool make_view_maps(CUtensorMap out[3], const void* base, int elem, const Geom& g, int BH,
-                    int d) {
+bool cached_maps(CUtensorMap* out, int n, int what, const void* base, int elem, const Geom& g,
+                 int BH, int d) {
   Key key;
   std::memset(&key, 0, sizeof(key));
   key.base = base;
+  key.what = what;
   key.elem = elem;
   key.T = g.T;
   key.l = g.l;
@@ -111,7 +130,7 @@ bool make_view_maps(CUtensorMap out[3], const void* base, int elem, const Geom& 
   for (int e = 0; e < kCacheSize; ++e) {
     if (g_cache[e].valid && g_cache[e].key == key) {
       g_cache[e].stamp = ++g_clock;
-      std::memcpy(out, g_cache[e].maps, sizeof(g_cache[e].maps));
+      std::memcpy(out, g_cache[e].maps, n * sizeof(CUtensorMap));
       return true;
     }
     // the first free slot, else the least recently used one
@@ -119,12 +138,25 @@ bool make_view_maps(CUtensorMap out[3], const void* base, int elem, const Geom& 
                        (!g_cache[e].valid || g_cache[e].stamp < g_cache[victim].stamp)))
       victim = e;
   }
-  if (!encode_views(out, base, elem, g, BH, d)) return false;
+  const bool ok = what == 0 ? encode_views(out, base, elem, g, BH, d)
+                            : encode_summary_rows(out, base, g, BH, d);
+  if (!ok) return false;
   g_cache[victim].key = key;
-  std::memcpy(g_cache[victim].maps, out, sizeof(g_cache[victim].maps));
+  std::memcpy(g_cache[victim].maps, out, n * sizeof(CUtensorMap));
   g_cache[victim].stamp = ++g_clock;
   g_cache[victim].valid = true;
   return true;
+}
+
+}  // namespace
+
+bool make_view_maps(CUtensorMap out[3], const void* base, int elem, const Geom& g, int BH,
+                    int d) {
+  return cached_maps(out, 3, 0, base, elem, g, BH, d);
+}
+
+bool make_summary_rows_map(CUtensorMap* out, const void* base, const Geom& g, int BH, int d) {
+  return cached_maps(out, 1, 1, base, ELEM_F32, g, BH, d);
 }
 
 int sm_count() {

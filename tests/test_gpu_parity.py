@@ -33,6 +33,13 @@ SMALL = [
     # divisors that are not powers of two in the kernels' index arithmetic:
     ("strided", "merged", 1, 2, 3072, 64, 8, 1, "bf16", 0.5),    # 384-row classes, 3 tiles each
     ("fixed", "merged", 3, 3, 1024, 64, 64, 8, "bf16", 0.5),     # 3 heads, 9 units per item
+    # natural key tiles of the merged fixed pattern stored directly with their
+    # summary rows accumulated: l > 128 (only a block's last tile has summary
+    # rows), 64 summary rows per tile (the most), and an l that does not
+    # divide 128 (whole tiles accumulate instead)
+    ("fixed", "merged", 1, 2, 4096, 64, 256, 16, "bf16", 0.5),
+    ("fixed", "merged", 1, 2, 1024, 64, 32, 16, "bf16", 0.5),
+    ("fixed", "merged", 1, 2, 1536, 64, 48, 8, "bf16", 0.5),
     # 18 heads of the fixed split pattern at std 0.5: the first key of a block
     # collects up to l query rows with large weights (max |dV| about 6); with P
     # rounded to bf16 before the dV product this case measured dV max-abs
