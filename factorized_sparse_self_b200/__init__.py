@@ -35,6 +35,7 @@ SIGNATURES = {
     "st_layout_counts": (ctypes.c_int, [_P, _P, _P]),
     "st_layout_segment_info": (ctypes.c_int, [_P, _i32, _i32, _P, _P, _P]),
     "st_layout_export": (ctypes.c_int, [_P, _i32, _i32, _i32, _P, _P, _P, _P, _P]),
+    "st_layout_rows": (ctypes.c_int, [_P, _i32, _i32, _P, _P]),
     "st_layout_nnz": (ctypes.c_int, [_P, _i32, _P]),
     "st_sparse_attn_fwd": (ctypes.c_int, [_P, ctypes.c_int, _i32, _i32, _i32, _i32,
                                           ctypes.c_float, _P, _P, _P, _P, _P, _P]),
@@ -154,6 +155,20 @@ class Layout:
         _check(lib().st_layout_launches(self.handle, dtype, ctypes.byref(f), ctypes.byref(b)),
                "st_layout_launches")
         return f.value, b.value
+
+    # row lists of st_layout_rows
+    ROWS_Q_ACC, ROWS_K_ACC, ROWS_Q_ZERO, ROWS_K_ZERO = 0, 1, 2, 3
+
+    def rows(self, hc, which):
+        """Natural rows of head class hc in row list `which` (st_layout_rows)."""
+        n = _i64(0)
+        _check(lib().st_layout_rows(self.handle, hc, which, None, ctypes.byref(n)),
+               "st_layout_rows")
+        out = np.zeros(max(n.value, 1), dtype=np.int32)
+        n2 = _i64(out.size)
+        _check(lib().st_layout_rows(self.handle, hc, which, out.ctypes.data_as(_P),
+                                    ctypes.byref(n2)), "st_layout_rows")
+        return out[:n.value]
 
     def export(self, hc, seg, transpose=False):
         """(ptr, idx, flags, live) numpy arrays of one segment (seg = -1: natural tiling)."""

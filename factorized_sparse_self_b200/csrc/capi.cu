@@ -250,6 +250,20 @@ st_status st_layout_nnz(const st_layout* L, int32_t hc, int64_t* nnz) {
   return ST_OK;
 }
 
+st_status st_layout_rows(const st_layout* L, int32_t hc, int32_t list, int32_t* rows,
+                         int64_t* count) {
+  if (!L || !count || hc < 0 || hc >= (int32_t)L->hcs.size() || list < 0 ||
+      list >= N_ROWLISTS)
+    return ST_ERR_INVALID;
+  const std::vector<int32_t>& r = L->rows[hc][list];
+  const int64_t cap = *count;
+  *count = (int64_t)r.size();
+  if (!rows) return ST_OK;
+  if (cap < (int64_t)r.size()) return ST_ERR_WORKSPACE;
+  if (!r.empty()) std::memcpy(rows, r.data(), sizeof(int32_t) * r.size());
+  return ST_OK;
+}
+
 st_status st_layout_export(const st_layout* L, int32_t hc, int32_t seg, int32_t transpose,
                            int32_t* ptr, int32_t* idx, uint8_t* flags, int32_t* live,
                            int64_t* sizes) {

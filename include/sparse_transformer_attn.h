@@ -130,6 +130,20 @@ st_status st_layout_export(const st_layout* layout, int32_t head_class, int32_t 
 /* Live pairs of one head of the class (sum over i of |S_i|). */
 st_status st_layout_nnz(const st_layout* layout, int32_t head_class, int64_t* nnz);
 
+/* Natural rows (positions t) of one head class that the 16-bit backward
+ * treats in a given way, ascending. list 0: dQ rows accumulated in fp32
+ * (several (key tile, query tile) pairs write them); 1: dK, dV rows
+ * accumulated in fp32; 2: dQ rows no pair writes (queries with an empty set:
+ * their gradient is zero and is zero-filled); 3: dK, dV rows no unit writes
+ * (keys in no query's set, zero-filled). Rows in no list are written
+ * directly in 16 bits. count_inout gives the capacity of rows (rows may be
+ * NULL: size query) and returns the number of rows. Host data only: works on
+ * layouts from st_pattern_layout_host. ST_ERR_INVALID for a bad head class or
+ * list, ST_ERR_WORKSPACE if the capacity is short (the count is still
+ * written). */
+st_status st_layout_rows(const st_layout* layout, int32_t head_class, int32_t list,
+                         int32_t* rows, int64_t* count_inout);
+
 /* Forward: O and LSE for all B*H heads ("Sparse Transformer" milestone page,
  * nlp-lineage, "The idea", "The notation": O_i = softmax(q_i K_{S_i}^T / sqrt(d))
  * V_{S_i}, normalised over S_i only, llm-arch-kb section 2, "Sparse attention

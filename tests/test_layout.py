@@ -4,6 +4,8 @@ The library computes tiles from closed-form row intervals; the oracle walks
 every live (i, j) pair. They must agree bit for bit: the same segments and
 views, the same tiles in the same order, the same live counts and flags.
 Runs on the CPU (host-only layouts, no CUDA call)."""
+import ctypes
+
 import numpy as np
 import pytest
 
@@ -117,3 +119,70 @@ def test_tile_coordinates_match_hand_derived_lists(orc, case):
     q, k, lv = _triples(ptr, idx, live, False)
     np.testing.assert_array_equal(np.stack([q, k, lv], axis=1), want)
     np.testing.assert_array_equal(flags, (want[:, 2] != 128 * 128).astype(np.uint8))
+
+
+# Which gradient rows the 16-bit backward zero-fills or accumulates in fp32
+# (st_layout_rows), against the sets themselves: the membership rule of the
+# oracle's numpy restatement, brute force over all (i, j) of one head.
+ROW_CASES = [
+    ("fixed", "merged", 1536, 128, 8),
+    ("fixed", "merged", 1024, 32, 16),
+    ("fixed", "merged", 2048, 256, 16),
+    ("fixed", "merged", 1536, 48, 8),
+    ("fixed", "split", 1024, 64, 8),
+    ("strided", "split", 1536, 192, 1),
+    ("strided", "merged", 2048, 256, 1),
+]
+
+
+@pytest.mark.parametrize("case", ROW_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_gradient_row_lists_follow_the_sets(case):
+    from oracle import reference_np as ref
+    kind, mode, T, l, c = case
+    L = st.st_pattern_layout_host(kind, mode, T, l, c)
+    n_hc = L.counts()[0]
+    for hc in range(n_hc):
+        m = ref.mask(kind, mode, T, l, c, hc)  # head hc has the class's parity
+        q_empty = set(np.flatnonzero(~m.any(axis=1)).tolist())
+        k_unused = set(np.flatnonzero(~m.any(axis=0)).tolist())
+        q_acc, k_acc = L.rows(hc, L.ROWS_Q_ACC), L.rows(hc, L.ROWS_K_ACC)
+        q_zero, k_zero = L.rows(hc, L.ROWS_Q_ZERO), L.rows(hc, L.ROWS_K_ZERO)
+        for r in (q_acc, k_acc, q_zero, k_zero):
+            assert np.all(np.diff(r) > 0) and (r.size == 0 or (r[0] >= 0 and r[-1] < T))
+        # a zero-filled row must have a zero gradient: no live pair at all
+        assert set(q_zero.tolist()) <= q_empty
+        assert set(k_zero.tolist()) <= k_unused
+        assert not set(q_zero.tolist()) & set(q_acc.tolist())
+        assert not set(k_zero.tolist()) & set(k_acc.tolist())
+    if kind == "fixed" and mode == "split":
+        # the summary heads read summary keys only: every other key row is
+        # zero-filled, and no summary key is
+        summary = np.flatnonzero(np.arange(T) % l >= l - c)
+        assert set(L.rows(1, L.ROWS_K_ZERO).tolist()) == set(range(T)) - set(summary.tolist())
+        assert L.rows(0, L.ROWS_K_ACC).size == 0  # block heads: one unit per key tile
+    if kind == "fixed" and mode == "merged":
+        summary = np.flatnonzero(np.arange(T) % l >= l - c)
+        if (128 % l == 0 and c * (128 // l) <= 64) or (l % 128 == 0 and c <= 64):
+            # block key tiles are stored directly and add only their summary
+            # rows: exactly the summary keys accumulate
+            assert np.array_equal(L.rows(0, L.ROWS_K_ACC), summary)
+        else:
+            # l does not divide 128: every block tile holds summary keys and
+            # accumulates as a whole
+            assert np.array_equal(L.rows(0, L.ROWS_K_ACC), np.arange(T))
+    if mode == "merged" or kind == "strided":
+        # causal sets are never empty: no dQ row is zero-filled
+        for hc in range(n_hc):
+            assert L.rows(hc, L.ROWS_Q_ZERO).size == 0
+
+
+def test_row_list_arguments():
+    L = st.st_pattern_layout_host("fixed", "merged", 1536, 128, 8)
+    with pytest.raises(st.StatusError):
+        L.rows(1, 0)  # one head class
+    with pytest.raises(st.StatusError):
+        L.rows(0, 4)
+    n = ctypes.c_int64(3)
+    buf = (ctypes.c_int32 * 3)()
+    assert st.lib().st_layout_rows(L.handle, 0, 1, buf, ctypes.byref(n)) == st.ST_ERR_WORKSPACE
+    assert n.value == 96  # 12 blocks x 8 summary keys, reported despite the short buffer
