@@ -341,31 +341,38 @@ def run_ours(args):
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
     d2h = sum(x.numel() * x.element_size() for x in (ho, hl, hdq, hdk, hdv))
 
-    # The batch entries go through the public API one at a time on two
-    # streams (each with its own backward workspace), so that the upload of
-    # entry b + 1 and the download of entry b - 1 overlap the compute of
-    # entry b (host-device copies run in both directions at once).
-    streams = [torch.cuda.Stream(device=dev) for _ in range(2)]
+    # The step goes through the public API in chunks of G heads of one batch
+    # entry (the head-range calls; about eight chunks per step), rotating over
+    # four streams with a backward workspace each, so that the uploads of
+    # later chunks and the downloads of earlier ones overlap the compute of
+    # the current one (host-device copies run in both directions at once).
+    n_streams = 4
+    target = max(1, (w.H * w.B) // 8)
+    G = max(g for g in range(1, w.H + 1) if w.H % g == 0 and g <= target)
+    chunks = [(b, h0) for b in range(w.B) for h0 in range(0, w.H, G)]
+    streams = [torch.cuda.Stream(device=dev) for _ in range(n_streams)]
     ws_b = [torch.empty(st.st_sparse_attn_bwd_workspace(L, dt_code, 1, w.H, w.T, w.d),
                         dtype=torch.uint8, device=dev) for _ in streams]
 
     def e2e_step():
         start = torch.cuda.Event()
         start.record(stream)
-        for b in range(w.B):
-            si = b % len(streams)
+        for n, (b, h0) in enumerate(chunks):
+            si = n % len(streams)
             sb = streams[si]
             sb.wait_event(start)
             with torch.cuda.stream(sb):
                 sl = slice(b, b + 1)
+                hs = slice(h0, h0 + G)
                 for hsrc, ddst in ((hq, qd), (hk, kd), (hv, vd), (hdo, dod)):
-                    ddst[sl].copy_(hsrc[sl], non_blocking=True)
-                st.st_sparse_attn_fwd(L, qd[sl], kd[sl], vd[sl], o=o[sl], lse=lse[sl], stream=sb)
+                    ddst[sl, hs].copy_(hsrc[sl, hs], non_blocking=True)
+                st.st_sparse_attn_fwd(L, qd[sl], kd[sl], vd[sl], o=o[sl], lse=lse[sl], stream=sb,
+                                      heads=(h0, G))
                 st.st_sparse_attn_bwd(L, qd[sl], kd[sl], vd[sl], o[sl], lse[sl], dod[sl],
                                       workspace=ws_b[si], dq=dq[sl], dk=dk[sl], dv=dv[sl],
-                                      stream=sb)
+                                      stream=sb, heads=(h0, G))
                 for dsrc, hdst in ((o, ho), (lse, hl), (dq, hdq), (dk, hdk), (dv, hdv)):
-                    hdst[sl].copy_(dsrc[sl], non_blocking=True)
+                    hdst[sl, hs].copy_(dsrc[sl, hs], non_blocking=True)
         for sb in streams:
             done = torch.cuda.Event()
             done.record(sb)
@@ -425,8 +432,9 @@ def run_ours(args):
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "how": "pinned host buffers; per batch entry: upload, forward, backward, "
-                       "download through the public API, entries alternating over two streams"},
+                "how": f"pinned host buffers; per chunk of {G} heads of one batch entry: "
+                       "upload, forward, backward, download through the public API (head-"
+                       f"range calls), {len(chunks)} chunks rotating over {n_streams} streams"},
         "gpu_launches": args.steps * (fl + bl),
         "clocks": clk.summary(),
     }
