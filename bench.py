@@ -547,9 +547,11 @@ def oracle_sample(w, budget_s=15.0):
     threads = len(os.sched_getaffinity(0))
 
     def run(nh):
+        """Seconds of one fwd + bwd over nh heads (the forward alone in run.fwd_s)."""
         args = [x[:, :nh].copy() for x in (qf, kf, vf, dof)]
         t0 = time.perf_counter()
         oracle.forward(w.kind, w.mode, args[0], args[1], args[2], w.l, w.c, threads=threads)
+        run.fwd_s = time.perf_counter() - t0
         oracle.backward(w.kind, w.mode, args[0], args[1], args[2], args[3], w.l, w.c,
                         threads=threads)
         return time.perf_counter() - t0
@@ -565,10 +567,12 @@ def oracle_sample(w, budget_s=15.0):
 def cpu_baseline(w, budget_s=15.0):
     run, nh, nnz, threads, _ = oracle_sample(w, budget_s=budget_s)
     t = run(nh)
+    tf = run.fwd_s
     return {"value": 14.0 * w.d * nnz / t / 1e12, "unit": "TFLOP/s", "cores": threads,
             "kind": "oracle",
             "sample": f"{nh} of {w.B * w.H} heads of {w.name}, full T, fwd + bwd, fp64 C++ "
-                      f"oracle, {t:.2f} s"}
+                      f"oracle, {t:.2f} s",
+            "fwd_value": 4.0 * w.d * nnz / tf / 1e12, "fwd_s": tf, "fwd_bwd_s": t}
 
 
 def run_reference(args):
