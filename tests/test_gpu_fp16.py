@@ -41,10 +41,13 @@ def test_fp16_parity_small(orc, case):
 @pytest.mark.parametrize("case", [
     ("fixed", "split", 4, 8, 4096, 64, 8, 64 ** -0.25),
     ("fixed", "merged", 2, 8, 12288, 128, 8, 0.5),
-], ids=["fixed-split-T4096", "fixed-merged-T12288"])
+    ("strided", "split", 4, 16, 12288, 192, 1, 0.5),
+    ("strided", "merged", 1, 8, 65536, 256, 1, 0.5),
+], ids=["fixed-split-T4096", "fixed-merged-T12288", "strided-split-T12288",
+        "strided-merged-T65536"])
 def test_fp16_full_size(orc, case):
-    """Two of the benchmark's shapes in fp16: every element of O, LSE, dQ, dK
-    and dV against the oracle fed the fp16-rounded inputs."""
+    """The benchmark's four 16-bit shapes in fp16: every element of O, LSE, dQ,
+    dK and dV against the oracle fed the fp16-rounded inputs."""
     kind, mode, B, H, T, l, c, std = case
     d = 64
     (q, k, v, do), (qd, kd, vd, dod) = device_inputs(B, H, T, d, "f16", std, seed=0)
