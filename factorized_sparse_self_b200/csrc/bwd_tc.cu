@@ -108,12 +108,21 @@ struct SmemBwd {
   int abort;
 };
 
+// PACKED: the layout packs short residue classes (Geom::cpt > 1); a separate
+// instantiation, so that other layouts' kernels carry none of its code.
+template <bool PACKED>
 __device__ __forceinline__ void load_tile(void* dst, const CUtensorMap* maps, int view,
                                           const Geom& g, int tile, int bh, uint64_t* bar) {
   if (view == VIEW_NAT) {
     tma_load_3d(dst, &maps[VIEW_NAT], bar, 0, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
     tma_load_4d(dst, &maps[VIEW_SUM], bar, 0, g.l - g.c, tile * g.sum_rows, bh);
+  } else if (PACKED) {
+    // packed short classes: one box of P rows per class, class after class
+    // (classes past l are zero-filled)
+    for (int k = 0; k < g.cpt; ++k)
+      tma_load_4d(static_cast<uint8_t*>(dst) + k * g.P * 128, &maps[VIEW_CLS], bar, 0,
+                  tile * g.cpt + k, 0, bh);
   } else {
     int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_load_4d(dst, &maps[VIEW_CLS], bar, 0, r, pb * kTile, bh);
@@ -121,12 +130,15 @@ __device__ __forceinline__ void load_tile(void* dst, const CUtensorMap* maps, in
 }
 
 // Prefetches a tile into L2 (the actual load follows when a ring stage frees).
+template <bool PACKED>
 __device__ __forceinline__ void prefetch_tile(const CUtensorMap* maps, int view, const Geom& g,
                                               int tile, int bh) {
   if (view == VIEW_NAT) {
     tma_prefetch_3d(&maps[VIEW_NAT], 0, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
     tma_prefetch_4d(&maps[VIEW_SUM], 0, g.l - g.c, tile * g.sum_rows, bh);
+  } else if (PACKED) {
+    for (int k = 0; k < g.cpt; ++k) tma_prefetch_4d(&maps[VIEW_CLS], 0, tile * g.cpt + k, 0, bh);
   } else {
     int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_prefetch_4d(&maps[VIEW_CLS], 0, r, pb * kTile, bh);
@@ -137,6 +149,7 @@ __device__ __forceinline__ void prefetch_tile(const CUtensorMap* maps, int view,
 // halves. (TMA copies issued by one thread are processed one after another,
 // copies of different threads in parallel: the two halves go out from two
 // lanes.)
+template <bool PACKED>
 __device__ __forceinline__ void reduce_half(const CUtensorMap* maps, int view, const Geom& g,
                                             int tile, int bh, const uint8_t* src, int h) {
   const uint8_t* s = src + h * kTileBytes;
@@ -144,6 +157,10 @@ __device__ __forceinline__ void reduce_half(const CUtensorMap* maps, int view, c
     tma_reduce_add_3d(&maps[VIEW_NAT], s, h * 32, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
     tma_reduce_add_4d(&maps[VIEW_SUM], s, h * 32, g.l - g.c, tile * g.sum_rows, bh);
+  } else if (PACKED) {
+    // packed short classes: one box per class (rows of classes past l are dropped)
+    for (int k = 0; k < g.cpt; ++k)
+      tma_reduce_add_4d(&maps[VIEW_CLS], s + k * g.P * 128, h * 32, tile * g.cpt + k, 0, bh);
   } else {
     int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_reduce_add_4d(&maps[VIEW_CLS], s, h * 32, r, pb * kTile, bh);
@@ -159,12 +176,16 @@ __device__ __forceinline__ void reduce_summary_rows(const CUtensorMap* map, cons
 }
 
 // Stores a 128-row bf16 tile (coordinates are never negative).
+template <bool PACKED>
 __device__ __forceinline__ void store_tile(const CUtensorMap* maps, int view, const Geom& g,
                                            int tile, int bh, const uint8_t* src) {
   if (view == VIEW_NAT) {
     tma_store_3d(&maps[VIEW_NAT], src, 0, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
     tma_store_4d(&maps[VIEW_SUM], src, 0, g.l - g.c, tile * g.sum_rows, bh);
+  } else if (PACKED) {
+    for (int k = 0; k < g.cpt; ++k)
+      tma_store_4d(&maps[VIEW_CLS], src + k * g.P * 128, 0, tile * g.cpt + k, 0, bh);
   } else {
     int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_store_4d(&maps[VIEW_CLS], src, 0, r, pb * kTile, bh);
@@ -207,7 +228,9 @@ __device__ __forceinline__ void live_rows(const Geom& g, int kview, int qview, i
       }
     }
   } else {
-    base = (qtile - fdiv(qtile, g.fpt) * g.ptiles) * kTile;
+    // query tile column x holds view row qtile * 128 + x; the key's class r
+    // starts at view row r * cw
+    base = qtile * kTile - (j - jb * l) * g.cw;
     lim = g.P;
     a = (rule == RULE_STRIDE) ? jb : jb + 2;
     b = lim;
@@ -231,7 +254,8 @@ __device__ __forceinline__ Unit unit_of(const BwdItem* items, int u, int NH, con
   return x;
 }
 
-template <bool F16>  // 16-bit element type: fp16 if true, else bf16
+// F16: 16-bit element type, fp16 if true, else bf16. PACKED: see load_tile.
+template <bool F16, bool PACKED>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __restrict__ items,
               int n_units, int NH, const QEnt* __restrict__ qents, Heads hs,
@@ -381,10 +405,10 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           // Q from lane 0, dO from lane 1; the L2 prefetches of the tile two
           // ahead from lanes 2, 3 (each thread's copies run one at a time)
           if (lane < 2)
-            load_tile(lane ? S.dout[s] : S.q[s], lane ? maps.dout : maps.q, x.it.qview, g,
+            load_tile<PACKED>(lane ? S.dout[s] : S.q[s], lane ? maps.dout : maps.q, x.it.qview, g,
                       qe.qtile, x.bh, &S.full[s]);
           else if (lane < 4 && pf >= 0)
-            prefetch_tile(lane == 3 ? maps.dout : maps.q, x.it.qview, g, pf, x.bh);
+            prefetch_tile<PACKED>(lane == 3 ? maps.dout : maps.q, x.it.qview, g, pf, x.bh);
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             const int row = lane + 32 * t;
@@ -408,7 +432,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           if (lane == 0) mbar_arrive_expect_tx(&S.kv_full[kb], 2 * kTileBytes);
           __syncwarp();
           if (lane < 2)  // K from lane 0, V from lane 1
-            load_tile(lane ? S.v[kb] : S.k[kb], lane ? maps.v : maps.k, y.it.kview, g,
+            load_tile<PACKED>(lane ? S.v[kb] : S.k[kb], lane ? maps.v : maps.k, y.it.kview, g,
                       y.it.ktile, y.bh, &S.kv_full[kb]);
           kv_last = m;
           return true;
@@ -566,9 +590,9 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         const bool w = mbar_wait(&S.stg_full, t & 1, wait_ns, abort);
         if (!__all_sync(0xffffffffu, w)) return false;
         if (pdirect) {
-          if (lane == 0) store_tile(maps.dqo, pv, g, ptile, pbh, S.stage);
+          if (lane == 0) store_tile<PACKED>(maps.dqo, pv, g, ptile, pbh, S.stage);
         } else if (lane < 2) {
-          reduce_half(maps.dq, pv, g, ptile, pbh, S.stage, lane);
+          reduce_half<PACKED>(maps.dq, pv, g, ptile, pbh, S.stage, lane);
         }
         if (lane < 2) {
           bulk_commit();
@@ -613,7 +637,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
         }
         if (x.it.kv_direct) {  // both 16-bit tiles in kvst
           if (lane < 2) {
-            store_tile(lane ? maps.dvo : maps.dko, x.it.kview, g, x.it.ktile, x.bh,
+            store_tile<PACKED>(lane ? maps.dvo : maps.dko, x.it.kview, g, x.it.ktile, x.bh,
                        S.kvst + lane * kTileBytes);
             bulk_commit();
           } else if (x.it.kv_direct == 2 && lane < 6) {
@@ -628,7 +652,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
           if (lane == 0) mbar_arrive(&S.dst_free);
         } else {  // lanes 0, 1: dV halves (in dst), read first; lanes 2, 3: dK halves
           if (lane < 4) {
-            reduce_half(lane < 2 ? maps.dv : maps.dk, x.it.kview, g, x.it.ktile, x.bh,
+            reduce_half<PACKED>(lane < 2 ? maps.dv : maps.dk, x.it.kview, g, x.it.ktile, x.bh,
                         lane < 2 ? S.dst : S.kvst, lane & 1);
             bulk_commit();
           }
@@ -960,8 +984,11 @@ cudaError_t tc_bwd_t(const Call& c, const void* q, const void* k, const void* v,
   cudaGetDevice(&dev);
   cudaError_t err = cudaSuccess;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    err = cudaFuncSetAttribute(bwd_tc_kernel<F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
+    err = cudaFuncSetAttribute(bwd_tc_kernel<F16, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(bwd_tc_kernel<F16, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
@@ -986,7 +1013,8 @@ cudaError_t tc_bwd_t(const Call& c, const void* q, const void* k, const void* v,
     zr.nk[hc] = L->dev.n_rows[hc][ROWS_K_ZERO];
   }
   record_begin(c);
-  bwd_tc_kernel<F16><<<grid, kThreads, smem, c.stream>>>(
+  auto kernel = L->geom.cpt > 1 ? bwd_tc_kernel<F16, true> : bwd_tc_kernel<F16, false>;
+  kernel<<<grid, kThreads, smem, c.stream>>>(
       maps, L->geom, (const BwdItem*)L->dev.bwd_split[f], (int)units, NH,
       (const QEnt*)L->dev.q_ents, heads_of(c), c.scale, c.scale * kLog2e, lse, D,
       zr, (uint4*)dq, (uint4*)dk, (uint4*)dv, sched_counter, slots, F16 ? 0 : nslots,

@@ -29,9 +29,10 @@ __device__ __forceinline__ int view_pos(const Geom& g, int v, int tile, int k) {
     const int q = fdiv(s, g.fc);
     return q * g.l + (g.l - g.c) + (s - q * g.c);
   }
-  int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
-  int p = pb * kTile + k;
-  if (p >= g.P) return -1;
+  // class view: view row y = r * cw + p
+  const int y = tile * kTile + k;
+  const int r = fdiv(y, g.fcw), p = y - r * g.cw;
+  if (p >= g.P || r >= g.l) return -1;
   return p * g.l + r;
 }
 

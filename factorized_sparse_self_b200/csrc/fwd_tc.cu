@@ -74,12 +74,21 @@ struct SmemFwd {
   int abort;
 };
 
+// PACKED: the layout packs short residue classes (Geom::cpt > 1); a separate
+// instantiation, so that other layouts' kernels carry none of its code.
+template <bool PACKED>
 __device__ __forceinline__ void load_tile(void* dst, const CUtensorMap* maps, int view,
                                           const Geom& g, int tile, int bh, uint64_t* bar) {
   if (view == VIEW_NAT) {
     tma_load_3d(dst, &maps[VIEW_NAT], bar, 0, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
     tma_load_4d(dst, &maps[VIEW_SUM], bar, 0, g.l - g.c, tile * g.sum_rows, bh);
+  } else if (PACKED) {
+    // packed short classes: one box of P rows per class, class after class
+    // (classes past l are zero-filled)
+    for (int k = 0; k < g.cpt; ++k)
+      tma_load_4d(static_cast<uint8_t*>(dst) + k * g.P * 128, &maps[VIEW_CLS], bar, 0,
+                  tile * g.cpt + k, 0, bh);
   } else {
     int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_load_4d(dst, &maps[VIEW_CLS], bar, 0, r, pb * kTile, bh);
@@ -87,12 +96,15 @@ __device__ __forceinline__ void load_tile(void* dst, const CUtensorMap* maps, in
 }
 
 // Prefetches a tile into L2 (the actual load follows when a ring stage frees).
+template <bool PACKED>
 __device__ __forceinline__ void prefetch_tile(const CUtensorMap* maps, int view, const Geom& g,
                                               int tile, int bh) {
   if (view == VIEW_NAT) {
     tma_prefetch_3d(&maps[VIEW_NAT], 0, tile * kTile, bh);
   } else if (view == VIEW_SUM) {
     tma_prefetch_4d(&maps[VIEW_SUM], 0, g.l - g.c, tile * g.sum_rows, bh);
+  } else if (PACKED) {
+    for (int k = 0; k < g.cpt; ++k) tma_prefetch_4d(&maps[VIEW_CLS], 0, tile * g.cpt + k, 0, bh);
   } else {
     int r = fdiv(tile, g.fpt), pb = tile - r * g.ptiles;
     tma_prefetch_4d(&maps[VIEW_CLS], 0, r, pb * kTile, bh);
@@ -128,8 +140,9 @@ __device__ __forceinline__ void live_cols(const Geom& g, const KeyEnt& ke, int i
     a = 0;
     b = blk * c + ((ke.rule == RULE_SUMMARY) ? max(0, off - (l - c) + 1) : 0);
   } else {
-    const int pb = ke.ktile - fdiv(ke.ktile, g.fpt) * g.ptiles;
-    base = pb * kTile;
+    // key tile column x holds view row ktile * 128 + x; the query's class r
+    // starts at view row r * cw
+    base = ke.ktile * kTile - (i - blk * l) * g.cw;
     lim = g.P;
     a = 0;
     b = (ke.rule == RULE_STRIDE) ? blk + 1 : blk - 1;
@@ -157,7 +170,7 @@ __device__ __forceinline__ Unit unit_of(const FwdItem* items, int u, int NH, con
 // the second pass of a two-pass layout and merges its result into the O and
 // LSE already in the outputs (a separate instantiation, so that one-pass
 // launches carry no merge code).
-template <bool F16, bool MERGE>
+template <bool F16, bool MERGE, bool PACKED>
 __global__ void __launch_bounds__(kThreads, 2)
 fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __restrict__ items,
               int n_units, int NH, const KeyEnt* __restrict__ keys, Heads hs,
@@ -273,7 +286,7 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           break;
         }
         mbar_arrive_expect_tx(&S.q_full[qb], kTileBytes);
-        load_tile(S.q[qb], maps.q, x.it.qview, g, x.it.qtile, x.bh, &S.q_full[qb]);
+        load_tile<PACKED>(S.q[qb], maps.q, x.it.qview, g, x.it.qtile, x.bh, &S.q_full[qb]);
         q_last[qb] = n;
         for (int e = x.it.kbeg; e < x.it.kend; ++e, ++gt) {
           const int s = gt % NS;
@@ -284,10 +297,10 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           if (force_timeout && gt == 0) continue;  // test hook: this stage never fills
           const KeyEnt ke = keys[e];
           mbar_arrive_expect_tx(&S.k_full[s], kTileBytes);
-          load_tile(S.k[s], maps.k, ke.kview, g, ke.ktile, x.bh, &S.k_full[s]);
+          load_tile<PACKED>(S.k[s], maps.k, ke.kview, g, ke.ktile, x.bh, &S.k_full[s]);
           if (e + 2 < x.it.kend) {
             const KeyEnt kn = keys[e + 2];
-            prefetch_tile(maps.k, kn.kview, g, kn.ktile, x.bh);
+            prefetch_tile<PACKED>(maps.k, kn.kview, g, kn.ktile, x.bh);
           }
           kv_last[s] = gt;
         }
@@ -327,10 +340,10 @@ fwd_tc_kernel(const __grid_constant__ FwdMaps maps, Geom g, const FwdItem* __res
           }
           const KeyEnt ke = keys[e];
           mbar_arrive_expect_tx(&S.v_full[s], kTileBytes);
-          load_tile(S.v[s], maps.v, ke.kview, g, ke.ktile, x.bh, &S.v_full[s]);
+          load_tile<PACKED>(S.v[s], maps.v, ke.kview, g, ke.ktile, x.bh, &S.v_full[s]);
           if (e + 2 < x.it.kend) {  // two tiles ahead of the ring: into L2 now
             const KeyEnt kn = keys[e + 2];
-            prefetch_tile(maps.v, kn.kview, g, kn.ktile, x.bh);
+            prefetch_tile<PACKED>(maps.v, kn.kview, g, kn.ktile, x.bh);
           }
           v_last[s] = gt;
         }
@@ -708,11 +721,12 @@ cudaError_t tc_fwd_t(const Call& c, const void* q, const void* k, const void* v,
   cudaGetDevice(&dev);
   cudaError_t err = cudaSuccess;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    err = cudaFuncSetAttribute(fwd_tc_kernel<F16, false>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err == cudaSuccess)
-      err = cudaFuncSetAttribute(fwd_tc_kernel<F16, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const void* ks[4] = {(const void*)fwd_tc_kernel<F16, false, false>,
+                         (const void*)fwd_tc_kernel<F16, true, false>,
+                         (const void*)fwd_tc_kernel<F16, false, true>,
+                         (const void*)fwd_tc_kernel<F16, true, true>};
+    for (int x = 0; x < 4 && err == cudaSuccess; ++x)
+      err = cudaFuncSetAttribute(ks[x], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
@@ -728,7 +742,10 @@ cudaError_t tc_fwd_t(const Call& c, const void* q, const void* k, const void* v,
     if (units > 0x7fffffff) return cudaErrorInvalidValue;
     const int grid = (int)std::min<long long>(units, 2LL * sms);
     // the second pass of a two-pass layout merges into the first's O, LSE
-    auto kernel = pass > 0 ? fwd_tc_kernel<F16, true> : fwd_tc_kernel<F16, false>;
+    const bool packed = L->geom.cpt > 1;
+    auto kernel = pass > 0 ? (packed ? fwd_tc_kernel<F16, true, true> : fwd_tc_kernel<F16, true, false>)
+                           : (packed ? fwd_tc_kernel<F16, false, true>
+                                     : fwd_tc_kernel<F16, false, false>);
     kernel<<<grid, kThreads, smem, c.stream>>>(
         maps, L->geom, (const FwdItem*)L->dev.fwd_items[pass], (int)units, NH,
         (const KeyEnt*)L->dev.key_ents, heads_of(c), scale_log2, (uint16_t*)o, lse,

@@ -88,7 +88,7 @@ bool rows_are_intervals(const SegDef& s, i64 T, i64 l) {
 i64 view_rows(uint8_t v, const Geom& g) {
   if (v == VIEW_NAT) return g.T;
   if (v == VIEW_SUM) return g.nsum;
-  return (i64)g.l * g.ptiles * kTile;  // padded classes
+  return (i64)g.l * g.cw;  // classes packed or padded to cw rows
 }
 
 typedef std::pair<i64, i64> Iv;
@@ -98,7 +98,7 @@ typedef std::pair<i64, i64> Iv;
 void row_intervals(const SegDef& s, const Geom& g, i64 i, std::vector<Iv>& out) {
   out.clear();
   const i64 l = g.l, c = g.c;
-  const i64 W = (i64)g.ptiles * kTile;
+  const i64 W = g.cw;
   auto push = [&](i64 a, i64 b) {
     if (b > a) out.push_back(Iv(a, b));
   };
@@ -146,7 +146,7 @@ void for_each_query_row(uint8_t qv, const Geom& g, F f) {
   if (qv == VIEW_NAT) {
     for (i64 t = 0; t < g.T; ++t) f(t, t);
   } else {
-    const i64 W = (i64)g.ptiles * kTile;
+    const i64 W = g.cw;
     for (i64 r = 0; r < g.l; ++r)
       for (i64 p = 0; p < g.P; ++p) f(r * W + p, p * g.l + r);
   }
@@ -207,8 +207,8 @@ void tile_rows(uint8_t v, const Geom& g, int32_t tile, std::vector<int32_t>& out
       const i64 sg = (i64)tile * kTile + k;
       if (sg < g.nsum) out.push_back((int32_t)((sg / g.c) * g.l + (g.l - g.c) + sg % g.c));
     } else {
-      const i64 r = tile / g.ptiles, p = (i64)(tile - r * g.ptiles) * kTile + k;
-      if (p < g.P) out.push_back((int32_t)(p * g.l + r));
+      const i64 y = (i64)tile * kTile + k, r = y / g.cw, p = y - r * g.cw;
+      if (r < g.l && p < g.P) out.push_back((int32_t)(p * g.l + r));
     }
   }
 }
@@ -334,12 +334,19 @@ st_status build_layout(const st_pattern_desc* desc, st_layout* L) {
   if (desc->kind != ST_DENSE_CAUSAL && has_cls(T, g.l)) {
     g.P = (int32_t)(T / g.l);
     g.ptiles = (g.P + kTile - 1) / kTile;
+    // (only the strided pattern uses the class view; the others keep cpt = 1
+    // so that their launches take the kernels without the packed paths)
+    const bool packed =
+        desc->kind == ST_STRIDED && g.P >= 8 && g.P <= 64 && kTile % g.P == 0;
+    g.cw = packed ? g.P : g.ptiles * kTile;
+    g.cpt = packed ? kTile / g.P : 1;
   }
   if (desc->kind == ST_FIXED && has_sum(T, g.l, c)) g.nsum = (int32_t)((T / g.l) * c);
   g.sum_rows = g.c >= 1 ? kTile / g.c : 0;
   g.fl = make_fastdiv(g.l);
   g.fc = make_fastdiv(g.c);
   g.fpt = make_fastdiv(g.ptiles);
+  g.fcw = make_fastdiv(g.cw);
 
   int nhc = (desc->kind != ST_DENSE_CAUSAL && mode == ST_HEADS_SPLIT) ? 2 : 1;
   L->hcs.assign((size_t)nhc, HeadClass());
@@ -491,7 +498,7 @@ void natural_tiles(const st_layout* L, int hc, std::vector<Tile>& out) {
   const Geom& g = L->geom;
   const HeadClass& H = L->hcs[(size_t)hc];
   const i64 nt = (g.T + kTile - 1) / kTile;
-  const i64 W = (i64)g.ptiles * kTile;
+  const i64 W = g.cw;
   out.clear();
   std::vector<i64> acc((size_t)nt, 0);
   std::vector<int32_t> touched;

@@ -140,10 +140,15 @@ struct Geom {
   int32_t T, l, c;
   int32_t P;       // rows per residue class, T / l (0 when no class view)
   int32_t ptiles;  // 128-row tiles per class, ceil(P / 128)
+  // Class-view rows: class r, row p is view row r * cw + p. Short classes
+  // (8 <= P <= 64, P dividing 128) are packed, cw = P and cpt = 128 / P whole
+  // classes per tile; otherwise each class is padded to cw = 128 * ptiles
+  // and cpt = 1.
+  int32_t cw, cpt;
   int32_t nsum;    // packed summary rows, (T / l) * c (0 when no summary view)
   int32_t kind, mode;
   int32_t sum_rows;      // summary-view rows of one 128-key tile per l-block, 128 / c
-  FastDiv fl, fc, fpt;   // division by l, c and ptiles
+  FastDiv fl, fc, fpt, fcw;  // division by l, c, ptiles and cw
 };
 
 // ---- host-side layout ------------------------------------------------------

@@ -57,7 +57,8 @@ bool encode_views(CUtensorMap out[3], const void* base, int elem, const Geom& g,
   if (g.P > 0) {
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)g.l, (cuuint64_t)(g.T / g.l), (cuuint64_t)BH};
     cuuint64_t str[3] = {row, (cuuint64_t)g.l * row, (cuuint64_t)g.T * row};
-    cuuint32_t box[4] = {inner, 1, (cuuint32_t)kTile, 1};
+    // packed short classes (cpt > 1) move one class of P rows per box
+    cuuint32_t box[4] = {inner, 1, (cuuint32_t)(g.cpt > 1 ? g.P : kTile), 1};
     if (enc(&out[VIEW_CLS], dt, 4, gp, dims, str, box, one, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)

@@ -370,8 +370,10 @@ void orc_backward_key_rows(int kind, int mode, i64 B, i64 H, i64 T, i64 d, i64 l
 //   view 0  natural order: position t;
 //   view 1  summary gather (keys only): the last c positions of every
 //           l-block, packed: sigma(j) = floor(j/l)*c + (j mod l) - (l-c);
-//   view 2  residue-class order: t = p*l + r is row p of class r; tiles never
-//           straddle two classes.
+//   view 2  residue-class order: t = p*l + r is row p of class r, view row
+//           r*W + p. Classes of P = T/l rows are padded to W = a multiple of
+//           128 rows, except short ones (8 <= P <= 64, P dividing 128), which
+//           are packed (W = P: 128/P whole classes per tile).
 // Tiles are 128 x 128 in view coordinates. This re-derivation walks every
 // (i, j) pair of the explicit sets, assigns it to its segment and counts the
 // pairs per tile; the library computes the same tiles from closed-form row
@@ -393,7 +395,7 @@ namespace {
 const i64 TILE = 128;
 
 struct ViewGeom {
-  i64 T, l, c, P, ptiles;
+  i64 T, l, c, P, ptiles, W;
 };
 
 bool has_cls(i64 T, i64 l) { return T % l == 0 && l < T; }
@@ -430,13 +432,13 @@ int seg_of(int kind, int mode, i64 l, i64 i, i64 j) {
 i64 view_ntiles(int view, const ViewGeom& g) {
   if (view == 0) return (g.T + TILE - 1) / TILE;
   if (view == 1) return ((g.T / g.l) * g.c + TILE - 1) / TILE;
-  return g.l * g.ptiles;
+  return (g.l * g.W + TILE - 1) / TILE;
 }
 
 i64 view_tile(int view, const ViewGeom& g, i64 t) {
   if (view == 0) return t / TILE;
   if (view == 1) return ((t / g.l) * g.c + (t % g.l) - (g.l - g.c)) / TILE;
-  return (t % g.l) * g.ptiles + (t / g.l) / TILE;
+  return ((t % g.l) * g.W + t / g.l) / TILE;
 }
 
 }  // namespace
@@ -456,10 +458,11 @@ void orc_segment_views(int kind, int mode, i64 T, i64 l, i64 c, int hc, int seg,
 // of the whole set (128 x 128 tiles of (i, j), no gather views).
 i64 orc_layout_tiles(int kind, int mode, i64 T, i64 l, i64 c, int hc, int seg, i64* qt, i64* kt,
                      i64* live, i64 cap) {
-  ViewGeom g{T, l, c, 0, 0};
+  ViewGeom g{T, l, c, 0, 0, 0};
   if (has_cls(T, l)) {
     g.P = T / l;
     g.ptiles = (g.P + TILE - 1) / TILE;
+    g.W = (g.P >= 8 && g.P <= 64 && TILE % g.P == 0) ? g.P : g.ptiles * TILE;
   }
   int qv = 0, kv = 0;
   if (seg >= 0) seg_views(kind, mode, T, l, c, hc, seg, &qv, &kv);
