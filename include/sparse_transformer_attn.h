@@ -89,7 +89,11 @@ typedef struct st_layout st_layout;
  * per key tile, its live query tiles (CSC), with a FULL/PARTIAL flag and the
  * live-pair count of every tile. Segments read keys in natural order, in
  * summary order (the last c positions of every block, packed) or in residue
- * order (positions p*l + r of one class r), so that their tiles are dense.
+ * order (position p*l + r at row p of class r, view row r*W + p), so that
+ * their tiles are dense. Residue classes of P = T/l rows are padded to W =
+ * 128*ceil(P/128) rows, except in strided layouts with 8 <= P <= 64 and P
+ * dividing 128, where W = P (128/P whole classes per 128-row tile). Tile t of
+ * a view covers view rows 128t .. 128t+127.
  * The device copy is uploaded with cudaMemcpyAsync on `stream`; the call
  * synchronises that stream once before returning. Runs once per shape.
  * Returns ST_ERR_INVALID for T < 1, l < 1, c outside [1, l] (fixed), or an
