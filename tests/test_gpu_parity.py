@@ -26,6 +26,9 @@ SMALL = [
     ("strided", "merged", 1, 2, 2048, 64, 256, 1, "bf16", 0.5),
     ("strided", "split", 1, 2, 1024, 64, 16, 1, "bf16", 0.5),    # 64-row classes, l << 128
     ("strided", "merged", 1, 2, 512, 64, 8, 1, "bf16", 0.5),
+    # residue classes packed 8 and 4 to a tile (P = 16, 32)
+    ("strided", "split", 1, 4, 1024, 64, 64, 1, "bf16", 0.5),
+    ("strided", "merged", 1, 2, 1024, 64, 32, 1, "bf16", 0.5),
     ("dense", "merged", 1, 2, 640, 64, 1, 1, "bf16", 0.5),
     ("strided", "merged", 1, 2, 256, 64, 300, 1, "bf16", 0.5),   # l > T: full causal
     ("strided", "split", 1, 2, 384, 64, 384, 1, "bf16", 0.5),    # l = T: A2 is the diagonal

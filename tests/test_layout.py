@@ -23,6 +23,10 @@ CASES = [
     ("strided", "merged", 2048, 256, 1),
     ("strided", "split", 1024, 16, 1),
     ("strided", "merged", 1024, 32, 1),
+    ("strided", "split", 1024, 64, 1),      # P = 16: classes packed 8 to a tile
+    ("strided", "merged", 512, 128, 1),     # P = 4: too short to pack, padded
+    ("strided", "split", 3072, 32, 1),      # P = 96 does not divide 128: padded
+    ("strided", "merged", 4096, 32, 1),     # P = 128: one class per tile
     ("strided", "merged", 1000, 48, 1),     # T not a multiple of l: no class view
     ("strided", "split", 384, 384, 1),      # l = T
     ("strided", "merged", 256, 1000, 1),    # l > T
