@@ -110,9 +110,10 @@ enum Elem : int { ELEM_BF16 = 0, ELEM_F16 = 1, ELEM_F32 = 2 };
 
 // Encodes the natural (3-D), summary and residue-class (4-D) TMA views of a
 // [B*H, T, d] tensor: 16-bit elements with 64-element boxes, or fp32 with
-// 32-element boxes; 128-byte swizzle; 128-row boxes. Views the layout lacks
-// get a copy of the natural map (never used). Returns false if the driver
-// rejects one.
+// 32-element boxes; 128-byte swizzle; 128-row boxes (in a layout that packs
+// short residue classes, Geom::cpt > 1, the class view's box is one class of
+// P rows). Views the layout lacks get a copy of the natural map (never used).
+// Returns false if the driver rejects one.
 bool make_view_maps(CUtensorMap out[3], const void* base, int elem, const Geom& g, int BH,
                     int d);
 
