@@ -246,11 +246,26 @@ struct Unit {
   int bh;
 };
 
-__device__ __forceinline__ Unit unit_of(const BwdItem* items, int u, int NH, const Heads& hs) {
+// Unit order: item-major (every head of the longest item first), or, when
+// the fp32 accumulator rows of all heads would not stay in L2, head-major
+// (all items of one head, longest first, then the next head).
+struct UnitOrder {
+  int head_major, n_items;
+  FastDiv fitems;
+};
+
+__device__ __forceinline__ Unit unit_of(const BwdItem* items, int u, int NH, const Heads& hs,
+                                        const UnitOrder& uo) {
   Unit x;
-  const int q = fdiv(u, hs.fnh);  // NH = the divisor of hs.fnh
-  x.it = items[q];
-  x.bh = head_of(u - q * NH, x.it.hclass, hs);
+  if (uo.head_major) {
+    const int h = fdiv(u, uo.fitems);
+    x.it = items[u - h * uo.n_items];
+    x.bh = head_of(h, x.it.hclass, hs);
+  } else {
+    const int q = fdiv(u, hs.fnh);  // NH = the divisor of hs.fnh
+    x.it = items[q];
+    x.bh = head_of(u - q * NH, x.it.hclass, hs);
+  }
   return x;
 }
 
@@ -258,7 +273,7 @@ __device__ __forceinline__ Unit unit_of(const BwdItem* items, int u, int NH, con
 template <bool F16, bool PACKED>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __restrict__ items,
-              int n_units, int NH, const QEnt* __restrict__ qents, Heads hs,
+              int n_units, int NH, UnitOrder uo, const QEnt* __restrict__ qents, Heads hs,
               float scale, float scale_log2, const float* __restrict__ lse,
               const float* __restrict__ Dg, ZeroRows zr, uint4* __restrict__ dq_out,
               uint4* __restrict__ dk_out, uint4* __restrict__ dv_out, int* sched_counter,
@@ -348,7 +363,7 @@ bwd_tc_kernel(const __grid_constant__ BwdMaps maps, Geom g, const BwdItem* __res
       auto valid = [&](int u, Unit& y) -> int {
         for (;;) {
           if (u >= n_units) return n_units;
-          y = unit_of(items, u, NH, hs);
+          y = unit_of(items, u, NH, hs, uo);
           if (y.bh >= 0) return u;
           int t = 0;
           if (lane == 0) t = atomicAdd(sched_counter, 1);
@@ -1004,6 +1019,16 @@ cudaError_t tc_bwd_t(const Call& c, const void* q, const void* k, const void* v,
   while (f < 2 && L->dev.max_split_len[f] > share) ++f;
   const long long units = (long long)L->dev.n_bwd_split[f] * NH;
   if (units > 0x7fffffff) return cudaErrorInvalidValue;
+  // fp32 accumulator rows all heads reduce into: head-major order when they
+  // exceed about the L2 (126 MB), so that one head's rows stay resident
+  double acc_bytes = 0.0;
+  for (int hc = 0; hc < (int)L->hcs.size(); ++hc)
+    acc_bytes += (double)(L->dev.n_rows[hc][ROWS_Q_ACC] + 2.0 * L->dev.n_rows[hc][ROWS_K_ACC]) *
+                 c.d * 4.0 * NH;
+  UnitOrder uo;
+  uo.head_major = acc_bytes > 128.0 * (1 << 20) ? 1 : 0;
+  uo.n_items = L->dev.n_bwd_split[f];
+  uo.fitems = make_fastdiv(uo.n_items);
   const int grid = (int)std::min<long long>(units, sms);
   ZeroRows zr;
   for (int hc = 0; hc < 2; ++hc) {
@@ -1015,7 +1040,7 @@ cudaError_t tc_bwd_t(const Call& c, const void* q, const void* k, const void* v,
   record_begin(c);
   auto kernel = L->geom.cpt > 1 ? bwd_tc_kernel<F16, true> : bwd_tc_kernel<F16, false>;
   kernel<<<grid, kThreads, smem, c.stream>>>(
-      maps, L->geom, (const BwdItem*)L->dev.bwd_split[f], (int)units, NH,
+      maps, L->geom, (const BwdItem*)L->dev.bwd_split[f], (int)units, NH, uo,
       (const QEnt*)L->dev.q_ents, heads_of(c), c.scale, c.scale * kLog2e, lse, D,
       zr, (uint4*)dq, (uint4*)dk, (uint4*)dv, sched_counter, slots, F16 ? 0 : nslots,
       c.status, c.wait_ns);
